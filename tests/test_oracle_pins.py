@@ -1,0 +1,349 @@
+"""Pins of the CPU oracle against facts that do not come from the oracle itself.
+
+Each pin is chosen so that a plausible slip (a dropped term, a wrong sign or index, a
+transposed operand, a wrong scale) fails at least one test:
+  * fp8 / bf16 decoding against torch's own dtype conversions, all codes;
+  * hand-worked golden values (tests/golden/*.json);
+  * closed forms (one-hot queries, ReLU(x) - ReLU(-x) = x, two-token softmax);
+  * special cases that reduce to a library routine (k >= L equals dense causal
+    attention, computed with torch's scaled_dot_product_attention in float64);
+  * invariants (paging, permutation, scaling) and brute-force rank counting.
+"""
+import json
+import math
+import os
+
+import numpy as np
+import pytest
+import torch
+
+from oracle import oracle as O
+
+GOLDEN = os.path.join(os.path.dirname(__file__), "golden")
+
+
+def _f(x):
+    return float("-inf") if x == "-inf" else float(x)
+
+
+def _bits(t: torch.Tensor) -> np.ndarray:
+    """Raw bytes of a bf16 / fp8 tensor as a numpy integer array."""
+    if t.dtype == torch.bfloat16:
+        return t.contiguous().view(torch.int16).numpy().view(np.uint16)
+    if t.dtype == torch.float8_e4m3fn:
+        return t.contiguous().view(torch.uint8).numpy()
+    return t.contiguous().numpy()
+
+
+# ---------------------------------------------------------------- dtype decoding
+def test_e4m3_all_codes_match_torch():
+    codes = torch.arange(256, dtype=torch.uint8)
+    ref = codes.view(torch.float8_e4m3fn).to(torch.float64).numpy()
+    got = np.array([O.e4m3_to_double(int(c)) for c in range(256)])
+    nan = np.isnan(ref)
+    assert np.array_equal(np.isnan(got), nan)
+    assert nan.sum() == 2  # S.1111.111 only
+    assert np.array_equal(got[~nan], ref[~nan])
+    assert got[0x7E] == 448.0 and got[0x01] == 2.0 ** -9
+
+
+def test_bf16_decode_matches_torch():
+    rng = np.random.default_rng(0)
+    bits = np.concatenate([rng.integers(0, 65536, 4000), [0, 0x8000, 0x7F80, 0x0001, 0x3F80]])
+    ref = torch.from_numpy(bits.astype(np.int16)).view(torch.bfloat16).double().numpy()
+    got = np.array([O.bf16_to_double(int(b)) for b in bits])
+    fin = np.isfinite(ref)
+    assert np.array_equal(got[fin], ref[fin])
+
+
+# ---------------------------------------------------------------- indexer
+def _run_indexer(q, w, k, k_scale, cu_q, seq_lens, page_size=64, q_dtype=O.F32, k_dtype=O.F32,
+                 q_scale=None, block_table=None, k_pages=None):
+    heads, dim = q.shape[1], q.shape[2]
+    L = int(max(seq_lens))
+    if k_pages is None:
+        n_pages = (k.shape[0] + page_size - 1) // page_size
+        k_pages = np.zeros((n_pages * page_size, dim), dtype=k.dtype)
+        k_pages[: k.shape[0]] = k
+        ks = np.ones(n_pages * page_size, dtype=np.float32)
+        if k_scale is not None:
+            ks[: k.shape[0]] = k_scale
+        block_table = np.arange(n_pages, dtype=np.int32)[None, :]
+    else:
+        ks = k_scale
+    return O.indexer_logits(q, q_dtype, q_scale, w, heads, dim, k_pages, k_dtype, ks, page_size,
+                            block_table, cu_q, seq_lens, L)
+
+
+def test_indexer_hand_golden():
+    g = json.load(open(os.path.join(GOLDEN, "indexer_hand.json")))
+    q = np.array(g["q"], dtype=np.float32)
+    w = np.array(g["w"], dtype=np.float32)
+    k = np.array(g["k"], dtype=np.float32)
+    out = _run_indexer(q, w, k, np.array(g["k_scale"], np.float32), g["cu_q"], g["seq_lens"])
+    exp = np.array([[_f(x) for x in r] for r in g["expected"]], dtype=np.float32)
+    assert np.array_equal(out, exp)
+
+
+def test_indexer_one_hot_closed_form():
+    """One head, w = 1, q = e_i: I[t, s] = ReLU(k[s, i]) * k_scale[s] -- no dot product."""
+    rng = np.random.default_rng(1)
+    L, dim = 70, 8
+    k = rng.standard_normal((L, dim)).astype(np.float32)
+    ks = rng.uniform(0.5, 2.0, L).astype(np.float32)
+    q = np.zeros((L, 1, dim), np.float32)
+    col = rng.integers(0, dim, L)
+    q[np.arange(L), 0, col] = 1.0
+    w = np.ones((L, 1), np.float32)
+    out = _run_indexer(q, w, k, ks, [0, L], [L])
+    for t in range(L):
+        exp = (np.maximum(k[: t + 1, col[t]].astype(np.float64), 0) * ks[: t + 1]).astype(np.float32)
+        assert np.array_equal(out[t, : t + 1], exp)
+        assert np.all(np.isneginf(out[t, t + 1:]))
+
+
+def test_indexer_relu_split_gives_textbook_dot():
+    """ReLU(x) - ReLU(-x) = x: I(q) - I(-q) is the plain dot product (numpy), one head."""
+    rng = np.random.default_rng(2)
+    L, dim = 40, 16
+    k = rng.standard_normal((L, dim)).astype(np.float32)
+    q = rng.standard_normal((L, 1, dim)).astype(np.float32)
+    w = np.ones((L, 1), np.float32)
+    a = _run_indexer(q, w, k, None, [0, L], [L]).astype(np.float64)
+    b = _run_indexer(-q, w, k, None, [0, L], [L]).astype(np.float64)
+    for t in range(L):
+        dot = k[: t + 1].astype(np.float64) @ q[t, 0].astype(np.float64)
+        np.testing.assert_allclose(a[t, : t + 1] - b[t, : t + 1], dot, rtol=1e-6, atol=1e-6)
+        assert np.all(a[t, : t + 1] >= 0) and np.all(b[t, : t + 1] >= 0)
+
+
+def test_indexer_weight_scale_and_head_permutation():
+    rng = np.random.default_rng(3)
+    L, H, dim = 50, 6, 8
+    k = rng.standard_normal((L, dim)).astype(np.float32)
+    q = rng.standard_normal((L, H, dim)).astype(np.float32)
+    w = rng.standard_normal((L, H)).astype(np.float32)
+    base = _run_indexer(q, w, k, None, [0, L], [L])
+    # scaling w by a power of two scales I exactly
+    assert np.array_equal(_run_indexer(q, 4 * w, k, None, [0, L], [L]), 4 * base)
+    # permuting heads jointly in q and w: same score up to summation order
+    p = rng.permutation(H)
+    perm = _run_indexer(q[:, p], w[:, p], k, None, [0, L], [L])
+    fin = np.isfinite(base)
+    np.testing.assert_allclose(perm[fin], base[fin], rtol=1e-6, atol=1e-6)
+    # q_scale multiplies the row
+    qs = rng.uniform(0.5, 2, L).astype(np.float32)
+    scaled = _run_indexer(q, w, k, None, [0, L], [L], q_scale=qs)
+    np.testing.assert_allclose(scaled[fin], (base * qs[:, None])[fin], rtol=1e-6, atol=1e-6)
+
+
+def test_indexer_paging_and_batch_positions():
+    """Logical order through a permuted block table, several sequences, last-nq queries."""
+    rng = np.random.default_rng(4)
+    page, dim, H = 4, 8, 3
+    lens, nq = [10, 7, 13], [3, 1, 13]
+    cu = np.concatenate([[0], np.cumsum(nq)]).astype(np.int32)
+    T = int(cu[-1])
+    keys = [rng.standard_normal((L, dim)).astype(np.float32) for L in lens]
+    q = rng.standard_normal((T, H, dim)).astype(np.float32)
+    w = rng.standard_normal((T, H)).astype(np.float32)
+    n_pages = sum((L + page - 1) // page for L in lens)
+    phys = rng.permutation(n_pages)
+    k_pages = np.full((n_pages * page, dim), np.nan, np.float32)  # unused rows poison
+    bt = np.full((3, 4), -1, np.int32)
+    off = 0
+    for b, L in enumerate(lens):
+        for lp in range((L + page - 1) // page):
+            bt[b, lp] = phys[off]
+            n = min(page, L - lp * page)
+            k_pages[phys[off] * page: phys[off] * page + n] = keys[b][lp * page: lp * page + n]
+            off += 1
+    out = _run_indexer(q, w, None, np.ones(n_pages * page, np.float32), cu, lens, page_size=page,
+                       block_table=bt, k_pages=k_pages)
+    for b, L in enumerate(lens):
+        single = _run_indexer(q[cu[b]:cu[b + 1]], w[cu[b]:cu[b + 1]], keys[b], None,
+                              [0, nq[b]], [L], page_size=page)
+        for i in range(nq[b]):
+            pos = L - nq[b] + i
+            assert np.array_equal(out[cu[b] + i, : pos + 1], single[i, : pos + 1])
+            assert np.all(np.isneginf(out[cu[b] + i, pos + 1:]))
+
+
+def test_indexer_fp8_inputs_match_decoded_values():
+    """fp8 codes (with scales) score like the same values decoded by torch in fp32."""
+    g = torch.Generator().manual_seed(5)
+    L, H, dim = 64, 4, 32
+    qf = torch.randn(L, H, dim, generator=g)
+    kf = torch.randn(L, dim, generator=g) * 3
+    q8, k8 = qf.to(torch.float8_e4m3fn), kf.to(torch.float8_e4m3fn)
+    ks = np.linspace(0.5, 1.5, L).astype(np.float32)
+    w = torch.randn(L, H, generator=g).numpy()
+    a = _run_indexer(_bits(q8).reshape(L, H, dim), w, _bits(k8), ks, [0, L], [L],
+                     q_dtype=O.E4M3, k_dtype=O.E4M3)
+    # the fp8 path reads codes: reshape keeps the byte array's shape semantics
+    b = _run_indexer(q8.float().numpy(), w, k8.float().numpy(), ks, [0, L], [L])
+    assert np.array_equal(a, b)
+
+
+# ---------------------------------------------------------------- top-k
+def test_topk_hand_golden():
+    g = json.load(open(os.path.join(GOLDEN, "topk_hand.json")))
+    for c in g["cases"]:
+        row = np.array([[_f(x) for x in c["row"]]], np.float32)
+        n = row.shape[1]
+        got = O.topk(row, [0, 1], [n], c["k"])
+        assert got[0].tolist() == c["expected"], c
+
+
+def _brute_topk(row, k):
+    """Selected iff fewer than k entries beat it (higher score, or equal score and lower index)."""
+    n = len(row)
+    sel = []
+    for i in range(n):
+        better = sum(1 for j in range(n) if row[j] > row[i] or (row[j] == row[i] and j < i))
+        if better < k:
+            sel.append(i)
+    return sel
+
+
+@pytest.mark.parametrize("seed", range(6))
+def test_topk_brute_force_rank(seed):
+    rng = np.random.default_rng(seed)
+    L, nq, k = 40, 40, 7
+    vals = rng.integers(-3, 4, (nq, L)).astype(np.float32)  # many ties
+    if seed % 2:
+        vals = rng.standard_normal((nq, L)).astype(np.float32)
+    got = O.topk(vals, [0, nq], [L], k)
+    for t in range(nq):
+        n = t + 1
+        exp = _brute_topk(vals[t, :n].tolist(), k)
+        assert got[t, : len(exp)].tolist() == exp
+        assert np.all(got[t, len(exp):] == -1)
+
+
+def test_topk_invariants_large_rows():
+    rng = np.random.default_rng(7)
+    L, k = 3000, 2048
+    rows = np.arange(0, L, 97)
+    vals = rng.standard_normal((len(rows), L)).astype(np.float32)
+    got = O.topk(vals, [0, L], [L], k, rows=rows)
+    for r, t in enumerate(rows):
+        n = t + 1
+        sel = got[r][got[r] >= 0]
+        assert len(sel) == min(k, n)
+        assert len(np.unique(sel)) == len(sel) and np.all(np.diff(sel) > 0)
+        assert sel.max() <= t
+        if n > k:
+            mask = np.zeros(n, bool)
+            mask[sel] = True
+            assert vals[r, :n][mask].min() >= vals[r, :n][~mask].max()
+
+
+# ---------------------------------------------------------------- sparse MLA
+def _mla(q, kv, idx, cu_q, seq_lens, scale, d_v, kv_scale=None, q_dtype=O.F32, kv_dtype=O.F32):
+    heads, d_qk = q.shape[1], q.shape[2]
+    L = int(max(seq_lens))
+    st = np.stack([np.arange(L, dtype=np.int32) + sum(seq_lens[:b]) for b in range(len(seq_lens))])
+    return O.sparse_mla(q, q_dtype, heads, d_qk, d_v, scale, kv, kv_dtype, kv_scale, 1, st, cu_q,
+                        seq_lens, idx)
+
+
+def test_mla_dense_equals_sdpa_when_k_ge_L():
+    """k >= L keeps every causal position: dense causal attention (torch SDPA, float64)."""
+    rng = np.random.default_rng(8)
+    L, nq, H, dqk, dv = 37, 11, 3, 20, 12
+    scale = 1 / math.sqrt(dqk)
+    q = rng.standard_normal((nq, H, dqk)).astype(np.float32)
+    kv = rng.standard_normal((L, dqk)).astype(np.float32)
+    idx = np.full((nq, 64), -1, np.int32)
+    for i in range(nq):
+        pos = L - nq + i
+        idx[i, : pos + 1] = rng.permutation(pos + 1)
+    out, lse = _mla(q, kv, idx, [0, nq], [L], scale, dv)
+    qt = torch.from_numpy(q).double().permute(1, 0, 2)           # [H, nq, dqk]
+    kt = torch.from_numpy(kv).double()[None].expand(H, L, dqk)
+    vt = torch.from_numpy(kv[:, :dv]).double()[None].expand(H, L, dv)
+    mask = torch.arange(L)[None, :] <= (L - nq + torch.arange(nq))[:, None]
+    ref = torch.nn.functional.scaled_dot_product_attention(qt, kt, vt, attn_mask=mask, scale=scale)
+    np.testing.assert_allclose(out, ref.permute(1, 0, 2).numpy(), rtol=1e-5, atol=1e-6)
+
+
+def test_mla_single_index_returns_value_row():
+    rng = np.random.default_rng(9)
+    L, H, dqk, dv = 16, 4, 10, 6
+    q = rng.standard_normal((L, H, dqk)).astype(np.float32)
+    kv = rng.standard_normal((L, dqk)).astype(np.float32)
+    idx = np.full((L, 3), -1, np.int32)
+    pick = np.array([rng.integers(0, t + 1) for t in range(L)])
+    idx[np.arange(L), 1] = pick
+    out, lse = _mla(q, kv, idx, [0, L], [L], 0.3, dv)
+    for t in range(L):
+        assert np.array_equal(out[t], np.broadcast_to(kv[pick[t], :dv], (H, dv)))
+        z = 0.3 * (q[t].astype(np.float64) @ kv[pick[t]].astype(np.float64))
+        np.testing.assert_allclose(lse[t], z, rtol=1e-6, atol=1e-6)
+
+
+def test_mla_two_token_logistic_closed_form():
+    """Two selected rows: o = sigmoid(z1 - z2) v1 + sigmoid(z2 - z1) v2."""
+    rng = np.random.default_rng(10)
+    H, dqk, dv, L = 2, 8, 5, 6
+    q = rng.standard_normal((1, H, dqk)).astype(np.float32)
+    kv = rng.standard_normal((L, dqk)).astype(np.float32)
+    idx = np.array([[4, -1, 1]], np.int32)
+    out, lse = _mla(q, kv, idx, [0, 1], [L], 0.5, dv)
+    for h in range(H):
+        z1 = 0.5 * float(q[0, h].astype(np.float64) @ kv[4].astype(np.float64))
+        z2 = 0.5 * float(q[0, h].astype(np.float64) @ kv[1].astype(np.float64))
+        a = 1 / (1 + math.exp(-(z1 - z2)))
+        exp = a * kv[4, :dv].astype(np.float64) + (1 - a) * kv[1, :dv].astype(np.float64)
+        np.testing.assert_allclose(out[0, h], exp, rtol=1e-6, atol=1e-6)
+        np.testing.assert_allclose(lse[0, h], max(z1, z2) + math.log1p(math.exp(-abs(z1 - z2))),
+                                   rtol=1e-6)
+
+
+def test_mla_permutation_identical_rows_and_lse_count():
+    rng = np.random.default_rng(11)
+    L, H, dqk, dv, k = 30, 3, 12, 8, 10
+    q = rng.standard_normal((L, H, dqk)).astype(np.float32)
+    kv = rng.standard_normal((L, dqk)).astype(np.float32)
+    idx = np.full((L, k), -1, np.int32)
+    for t in range(L):
+        n = min(k, t + 1)
+        idx[t, :n] = rng.choice(t + 1, n, replace=False)
+    a, la = _mla(q, kv, idx, [0, L], [L], 0.2, dv)
+    perm = np.stack([rng.permutation(k) for _ in range(L)])
+    b, lb = _mla(q, kv, np.take_along_axis(idx, perm, 1), [0, L], [L], 0.2, dv)
+    np.testing.assert_allclose(a, b, rtol=1e-6, atol=1e-7)
+    # identical KV rows: output is that row and lse = z + log(n)
+    same = np.broadcast_to(kv[:1], kv.shape).copy()
+    c, lc = _mla(q, same, idx, [0, L], [L], 0.2, dv)
+    for t in range(L):
+        n = min(k, t + 1)
+        np.testing.assert_allclose(c[t], np.broadcast_to(same[0, :dv], (H, dv)), rtol=1e-6,
+                                   atol=1e-7)
+        z = 0.2 * (q[t].astype(np.float64) @ same[0].astype(np.float64))
+        np.testing.assert_allclose(lc[t], z + math.log(n), rtol=1e-6, atol=1e-6)
+
+
+def test_mla_fp8_kv_and_bf16_q_match_decoded_values():
+    g = torch.Generator().manual_seed(12)
+    L, H, dqk, dv = 20, 4, 24, 16
+    q = torch.randn(L, H, dqk, generator=g).to(torch.bfloat16)
+    kvf = torch.randn(L, dqk, generator=g)
+    amax = kvf.abs().amax(1)
+    sc = (amax / 448).float()
+    k8 = (kvf / sc[:, None]).clamp(-448, 448).to(torch.float8_e4m3fn)
+    idx = np.stack([np.r_[np.arange(t + 1), -np.ones(L - t - 1)] for t in range(L)]).astype(np.int32)
+    a, la = _mla(_bits(q).reshape(L, H, dqk), _bits(k8), idx, [0, L], [L], 0.25, dv,
+                 kv_scale=sc.numpy(), q_dtype=O.BF16, kv_dtype=O.E4M3)
+    deq = (k8.double() * sc.double()[:, None]).float().numpy()
+    b, lb = _mla(q.float().numpy(), deq, idx, [0, L], [L], 0.25, dv)
+    np.testing.assert_allclose(a, b, rtol=1e-5, atol=1e-6)
+    np.testing.assert_allclose(la, lb, rtol=1e-5, atol=1e-6)
+
+
+def test_mla_rejects_noncausal_index():
+    q = np.zeros((1, 1, 4), np.float32)
+    kv = np.zeros((4, 4), np.float32)
+    with pytest.raises(ValueError):
+        _mla(q, kv, np.array([[3]], np.int32), [0, 1], [3], 1.0, 2)
