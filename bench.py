@@ -1,0 +1,453 @@
+#!/usr/bin/env python
+"""DSA hot-path throughput on B200 through libdsa's C ABI.
+
+One step = one pass of the whole hot path (Lightning Indexer logits -> top-k ->
+sparse MLA (+ split merge)) over one batch of synthetic input.  The default workload
+is decode: 32 sequences x 8192 context, one query each, FP8 indexer 64 x 128 (page
+64), top-k 2048, 128-head MLA over bf16 576-d latent KV (page 1).
+
+Timing: W untimed warm-up steps, then exactly K timed steps of the fused call
+(dsa_decode / the prefill sequence), each bracketed by CUDA events on the launching
+stream, with a 256 MiB write between steps to flush L2 (inputs here are ~120 MB,
+below the 126 MB L2).  A second K-step loop times the same kernels stage by stage
+for the roofline.  Multi-GPU runs are independent replicas (one batch per rank, no
+data-path collective): value = all ranks' tokens / the slowest rank's time.
+
+`--impl reference` times the CPU oracle on a bounded sample of the same workload.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import long_context_sparse_fp8_b200 as L  # noqa: E402
+from long_context_sparse_fp8_b200 import workloads as W  # noqa: E402
+
+METRIC = "DSA tokens/s (decode & prefill) on 1 B200; % of HBM / tensor-core roofline"
+FLUSH_BYTES = 256 << 20
+
+WORKLOADS = {
+    "decode_b32_ctx8192": (W.decode_b32_8k, "decode"),
+    "prefill_L32768_q8192": (W.prefill_32k, "prefill"),
+    "decode_b64_ctx64k-128k_fp8kv": (W.decode_b64_128k, "decode"),
+}
+
+
+def parse():
+    p = argparse.ArgumentParser()
+    p.add_argument("--gpus", type=int, default=1)
+    p.add_argument("--steps", type=int, default=20)
+    p.add_argument("--warmup", type=int, default=5)
+    p.add_argument("--impl", choices=["dsa", "reference"], default="dsa")
+    p.add_argument("--workload", choices=sorted(WORKLOADS), default="decode_b32_ctx8192")
+    p.add_argument("--no-cpu-baseline", action="store_true")
+    p.add_argument("--cpu-seconds", type=float, default=12.0)
+    return p.parse_args()
+
+
+# ----------------------------------------------------------------------------- plumbing
+def dist_setup(args):
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+        torch.cuda.set_device(local)
+        torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+    else:
+        torch.cuda.set_device(0)
+    return rank, world
+
+
+def barrier(world):
+    if world > 1:
+        torch.distributed.barrier()
+    torch.cuda.synchronize()
+
+
+def max_over_ranks(x: float, world: int) -> float:
+    if world == 1:
+        return x
+    t = torch.tensor([x], device="cuda", dtype=torch.float64)
+    torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+    return float(t.item())
+
+
+class ClockSampler:
+    """nvidia-smi clocks / throttle reasons sampled every 200 ms during the timed loop."""
+    Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+         "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+         "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.gpu}", f"--query-gpu={self.Q}",
+                 "--format=csv,noheader,nounits", "-lms", "200"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except (OSError, FileNotFoundError):
+            self.proc = None
+        return self
+
+    def __exit__(self, *exc):
+        self.lines = []
+        if self.proc is not None:
+            time.sleep(0.25)
+            self.proc.terminate()
+            try:
+                out, _ = self.proc.communicate(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+                out, _ = self.proc.communicate()
+            self.lines = [ln for ln in out.splitlines() if ln.strip()]
+
+    def summary(self):
+        sm, smax, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in getattr(self, "lines", []):
+            f = [x.strip() for x in ln.split(",")]
+            if len(f) < 9:
+                continue
+            try:
+                sm.append(float(f[1]))
+                smax = float(f[2])
+            except ValueError:
+                continue
+            for n, v in zip(names, f[5:9]):
+                if v.lower().startswith("active"):
+                    reasons.add(n)
+        if not sm:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unsampled"]}
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": smax, "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+def measured_peaks():
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            d = json.load(f)
+        return d["hbm_gbs"], d["bf16_tflops"], "measured"
+    except (OSError, KeyError, ValueError):
+        return 6650.0, 1590.0, "fallback"
+
+
+def ncu_traffic(kernel_file: str):
+    """DRAM bytes per launch from the committed ncu summary, if the kernel is unchanged."""
+    path = os.path.join(ROOT, "profiles", "ncu_traffic.json")
+    try:
+        with open(path) as f:
+            rec = json.load(f)
+    except (OSError, ValueError):
+        return None
+    src = os.path.join(ROOT, "long_context_sparse_fp8_b200", "csrc", kernel_file)
+    try:
+        sha = hashlib.sha256(open(src, "rb").read()).hexdigest()[:16]
+    except OSError:
+        return None
+    entry = rec.get(kernel_file)
+    if not entry or entry.get("source_sha") != sha:
+        return None
+    return entry.get("dram_bytes_per_launch")
+
+
+# ----------------------------------------------------------------------------- workload
+class Step:
+    """Buffers and calls of one hot-path step on one GPU."""
+
+    def __init__(self, wl: W.Workload, mode: str):
+        s = wl.spec
+        self.wl, self.mode, self.s = wl, mode, s
+        self.batch = L.Batch(wl.cu_q, wl.seq_lens, s.total_q, s.max_seq_len)
+        self.kc = L.PagedCache(wl.k_pages, wl.k_block_table, W.INDEXER_PAGE, wl.k_scale)
+        self.kv = L.PagedCache(wl.kv, wl.kv_slot_table, 1, wl.kv_scale)
+        dev = wl.device
+        self.ld = (s.max_seq_len + 63) // 64 * 64
+        self.logits = torch.empty(s.total_q, self.ld, device=dev)
+        self.idx = torch.empty(s.total_q, s.topk, dtype=torch.int32, device=dev)
+        self.out = torch.empty(s.total_q, s.heads, s.d_v, dtype=torch.bfloat16, device=dev)
+        self.lse = torch.empty(s.total_q, s.heads, device=dev)
+        n = L.dsa_decode_workspace_size(self.batch, s.topk, s.heads, s.d_v)
+        self.ws = torch.empty(max(n, 16), dtype=torch.uint8, device=dev)
+        m = L.dsa_sparse_mla_decode_workspace_size(s.total_q, s.heads, s.d_v, s.topk)
+        self.mla_ws = torch.empty(max(m, 16), dtype=torch.uint8, device=dev)
+        self.has_combine = m > 0   # the decode MLA splits each row's list and merges
+
+    def fused(self):
+        s = self.s
+        if self.mode == "decode":
+            L.dsa_decode(self.wl.q_idx, None, self.wl.w, self.kc, s.topk, self.wl.q, self.kv,
+                         self.batch, s.d_v, s.softmax_scale, self.out, self.lse, self.idx,
+                         self.ws)
+        else:
+            for f in self.stages():
+                f()
+
+    def stages(self):
+        s, wl = self.s, self.wl
+        mla = (lambda: L.dsa_sparse_mla_decode(wl.q, self.kv, self.batch, self.idx, s.d_v,
+                                               s.softmax_scale, self.out, self.lse, self.mla_ws)) \
+            if self.mode == "decode" else \
+            (lambda: L.dsa_sparse_mla_prefill(wl.q, self.kv, self.batch, self.idx, s.d_v,
+                                              s.softmax_scale, self.out, self.lse))
+        return [lambda: L.dsa_indexer_logits(wl.q_idx, None, wl.w, self.kc, self.batch,
+                                             self.logits),
+                lambda: L.dsa_topk(self.logits, self.batch, s.topk, self.idx),
+                mla]
+
+    def launches_per_step(self) -> int:
+        combine = 1 if (self.mode == "decode" and self.has_combine) else 0
+        return 3 + combine
+
+    # algorithmic bytes / flops per stage (what the method must touch)
+    def work(self):
+        s, wl = self.s, self.wl
+        T, k = s.total_q, s.topk
+        pos = []
+        for b in range(s.num_seqs):
+            for i in range(s.nq[b]):
+                pos.append(s.seq_lens[b] - s.nq[b] + i)
+        n_pairs = sum(p + 1 for p in pos)                     # causal (query, key) pairs
+        keys_read = sum(s.seq_lens) if self.mode == "decode" else s.max_seq_len * s.num_seqs
+        idx_bytes_key = s.idx_dim * (1 if s.idx_fp8 else 4) + 4
+        n_sel = sum(min(k, p + 1) for p in pos)
+        kv_row = s.d_qk * (1 if s.kv_fp8 else 2) + (4 if s.kv_fp8 else 0)
+        q_bytes = T * s.heads * s.d_qk * 2
+        o_bytes = T * s.heads * s.d_v * 2
+        return {
+            "indexer": {"bytes": keys_read * idx_bytes_key + T * s.idx_heads * (s.idx_dim + 4)
+                        + n_pairs * 4,
+                        "flops": 2 * n_pairs * s.idx_heads * s.idx_dim},
+            "topk": {"bytes": n_pairs * 4 + T * k * 4, "flops": 0},
+            "mla": {"bytes": n_sel * (kv_row + 8) + q_bytes + o_bytes + T * s.heads * 4,
+                    "flops": 2 * n_sel * s.heads * (s.d_qk + s.d_v)},
+        }
+
+
+def timed_loop(fn_list, steps, flush, stream):
+    """K steps; before each, a 256 MiB write flushes L2; events around every stage."""
+    evs = []
+    for _ in range(steps):
+        flush.zero_()
+        e = [torch.cuda.Event(enable_timing=True) for _ in range(len(fn_list) + 1)]
+        e[0].record(stream)
+        for j, f in enumerate(fn_list):
+            f()
+            e[j + 1].record(stream)
+        evs.append(e)
+    torch.cuda.synchronize()
+    return [[e[j].elapsed_time(e[j + 1]) for j in range(len(fn_list))] for e in evs]
+
+
+def run_dsa(args, rank, world):
+    spec_fn, mode = WORKLOADS[args.workload]
+    spec = spec_fn()
+    spec.seed += 1000 * rank  # independent replica inputs per rank
+    dev = torch.device("cuda", torch.cuda.current_device())
+    wl = W.make(spec, device=dev)
+    st = Step(wl, mode)
+    stream = torch.cuda.current_stream()
+    flush = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device=dev)
+
+    for _ in range(max(3, args.warmup)):
+        st.fused()
+    torch.cuda.synchronize()
+    if L.dsa_device_check() != 0:
+        raise RuntimeError("device check recorded an error during warm-up")
+
+    # ---- headline: K fused steps
+    barrier(world)
+    with ClockSampler(torch.cuda.current_device()) as clk:
+        step_ms = [sum(x) for x in timed_loop([st.fused], args.steps, flush, stream)]
+    barrier(world)
+    ms = statistics.mean(step_ms)
+    ms_max = max_over_ranks(ms, world)
+    tokens = spec.total_q
+    value = tokens * world / (ms_max / 1e3)
+
+    # ---- per-stage breakdown of the same kernels (roofline)
+    barrier(world)
+    stage_ms = timed_loop(st.stages(), args.steps, flush, stream)
+    barrier(world)
+    names = ["indexer", "topk", "mla"]
+    mean_stage = {n: statistics.mean(r[j] for r in stage_ms) for j, n in enumerate(names)}
+    work = st.work()
+    hbm_gbs, bf16_tf, peak_kind = measured_peaks()
+    dom = max(mean_stage, key=mean_stage.get)
+    if mode == "decode" or dom == "topk":
+        achieved = work[dom]["bytes"] / (mean_stage[dom] / 1e3) / 1e9
+        roof = {"bound": "hbm", "achieved": round(achieved, 1), "peak": hbm_gbs, "unit": "GB/s"}
+    else:
+        fl = work[dom]["flops"] / (mean_stage[dom] / 1e3) / 1e12
+        peak = bf16_tf * (2.0 if dom == "indexer" else 1.0)
+        roof = {"bound": "tensor", "achieved": round(fl, 1), "peak": peak, "unit": "TFLOP/s"}
+    roof["frac"] = round(roof["achieved"] / roof["peak"], 4)
+    kernel_file = {"indexer": "indexer_generic.cu", "topk": "topk.cu",
+                   "mla": "mla_generic.cu"}[dom]
+    roof["traffic"] = ncu_traffic(kernel_file)
+    roof["kernel"] = dom
+    roof["peak_source"] = f"{peak_kind} ({'burst' if roof['unit'] == 'GB/s' else 'burst bf16'})"
+    roof["stage_ms"] = {n: round(v, 4) for n, v in mean_stage.items()}
+    roof["algorithmic_bytes_per_launch"] = work[dom]["bytes"]
+
+    # ---- end to end through host buffers (pinned H2D of the step's queries, D2H of o)
+    e2e = None
+    if mode == "decode":
+        h_qidx = wl.q_idx.cpu().pin_memory()
+        h_w = wl.w.cpu().pin_memory()
+        h_q = wl.q.cpu().pin_memory()
+        h_out = torch.empty(st.out.shape, dtype=st.out.dtype).pin_memory()
+
+        def e2e_step():
+            wl.q_idx.copy_(h_qidx, non_blocking=True)
+            wl.w.copy_(h_w, non_blocking=True)
+            wl.q.copy_(h_q, non_blocking=True)
+            st.fused()
+            h_out.copy_(st.out, non_blocking=True)
+
+        for _ in range(3):
+            e2e_step()
+        barrier(world)
+        e_ms = statistics.mean(sum(x) for x in timed_loop([e2e_step], args.steps, flush, stream))
+        e_ms = max_over_ranks(e_ms, world)
+        h2d = sum(t.numel() * t.element_size() for t in (h_qidx, h_w, h_q))
+        e2e = {"value": round(tokens * world / (e_ms / 1e3), 1), "unit": "tokens/s",
+               "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": h_out.numel() * 2,
+               "ms_per_step": round(e_ms, 4)}
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        cpu = cpu_baseline(wl, mode, args.cpu_seconds)
+        cpu["kind"] = "oracle"
+
+    if L.dsa_device_check() != 0:
+        raise RuntimeError("device check recorded an error in the timed region")
+    return {
+        "metric": METRIC, "value": round(value, 1), "unit": "tokens/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms_max, 5),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "fp8 e4m3 (indexer) + bf16 (MLA), fp32 accumulate",
+        "data": "synthetic (seeded N(0,1) caches and queries)",
+        "config": {"workload": spec.name, "mode": mode, "num_seqs": spec.num_seqs,
+                   "context": spec.max_seq_len, "queries": spec.total_q, "topk": spec.topk,
+                   "indexer": f"{'fp8 e4m3' if spec.idx_fp8 else 'fp32'} {spec.idx_heads}x"
+                              f"{spec.idx_dim}, page 64, per-token scale",
+                   "mla": f"{spec.heads} heads, d_qk {spec.d_qk}, d_v {spec.d_v}, "
+                          f"{'fp8' if spec.kv_fp8 else 'bf16'} latent KV page 1",
+                   "l2": "flushed between steps (256 MiB write)",
+                   "parallelism": f"replicas x{world}"},
+        "roofline": roof, "cpu_baseline": cpu, "e2e": e2e, "clocks": clk.summary(),
+        "gpu_launches": st.launches_per_step() * args.steps,
+    }
+
+
+# ----------------------------------------------------------------------------- oracle arm
+def _oracle_rows(wl, mode, rows):
+    sys.path.insert(0, os.path.join(ROOT, "tests"))
+    import _helpers as H
+    from oracle import oracle as O
+    logits = H.oracle_logits(wl, rows)
+    cu = H.np_bits(wl.cu_q)
+    lens = H.np_bits(wl.seq_lens)
+    sel = O.topk(logits, cu, lens, wl.spec.topk, rows=rows)
+    H.oracle_mla(wl, sel, rows)
+
+
+def cpu_baseline(wl, mode, seconds):
+    """The oracle, as it stands, on a bounded row sample of the same workload."""
+    import numpy as np
+    from oracle import oracle as O
+    T = wl.spec.total_q
+    t0 = time.perf_counter()
+    _oracle_rows(wl, mode, np.array([T - 1]))
+    one = time.perf_counter() - t0
+    threads = O.num_threads()
+    n = int(max(1, min(T, seconds / max(one, 1e-3) * threads)))
+    rows = np.linspace(0, T - 1, n).round().astype(np.int64)
+    rows = np.unique(rows)
+    t0 = time.perf_counter()
+    _oracle_rows(wl, mode, rows)
+    dt = time.perf_counter() - t0
+    return {"value": round(len(rows) / dt, 3), "unit": "tokens/s", "cores": threads,
+            "sample": f"{len(rows)} of {T} query rows of {wl.spec.name} (indexer + top-k + MLA "
+                      f"per row, fp64), {dt:.1f} s"}
+
+
+def run_reference(args, rank, world):
+    if rank != 0:
+        return None
+    import numpy as np
+    from oracle import oracle as O
+    spec_fn, mode = WORKLOADS[args.workload]
+    spec = spec_fn()
+    dev = "cuda" if torch.cuda.is_available() else "cpu"
+    wl = W.make(spec, device=dev)
+    T = spec.total_q
+    # size each step's sample so the whole run stays within a few minutes
+    t0 = time.perf_counter()
+    _oracle_rows(wl, mode, np.array([T - 1]))
+    one = time.perf_counter() - t0
+    threads = O.num_threads()
+    budget = 150.0 / max(1, args.steps + args.warmup)
+    per_step = int(max(1, min(T, budget / max(one, 1e-3) * threads)))
+    rng = np.random.default_rng(0)
+    for _ in range(args.warmup):
+        _oracle_rows(wl, mode, np.sort(rng.choice(T, per_step, replace=False)))
+    times = []
+    for _ in range(args.steps):
+        rows = np.sort(rng.choice(T, per_step, replace=False))
+        t0 = time.perf_counter()
+        _oracle_rows(wl, mode, rows)
+        times.append(time.perf_counter() - t0)
+    ms = statistics.mean(times) * 1e3
+    value = per_step / (ms / 1e3)
+    sample = (f"{per_step} of {T} query rows per step of {spec.name} (indexer + top-k + MLA, "
+              f"fp64)")
+    return {
+        "impl": "reference", "metric": METRIC, "value": round(value, 3), "unit": "tokens/s",
+        "n_gpus": world, "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms, 3),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "f64", "data": "synthetic (seeded N(0,1) caches and queries)",
+        "config": {"workload": spec.name, "mode": mode, "queries": T, "topk": spec.topk},
+        "cpu_baseline": {"kind": "oracle", "cores": threads, "sample": sample,
+                         "value": round(value, 3), "unit": "tokens/s"},
+        "e2e": {"value": round(value, 3), "unit": "tokens/s", "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }
+
+
+def main():
+    args = parse()
+    if args.impl == "reference":
+        rank = int(os.environ.get("RANK", "0"))
+        world = int(os.environ.get("WORLD_SIZE", "1"))
+        res = run_reference(args, rank, world)
+        if res is not None:
+            print(json.dumps(res), flush=True)
+        return
+    rank, world = dist_setup(args)
+    try:
+        res = run_dsa(args, rank, world)
+        if rank == 0:
+            print(json.dumps(res), flush=True)
+    finally:
+        if world > 1:
+            torch.distributed.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,45 @@
+// kernels.h -- internal launchers of libdsa (host side, C++).  The public C ABI
+// in include/dsa.h validates arguments and then calls these.
+#pragma once
+
+#include <cuda_runtime.h>
+
+#include "common.cuh"
+
+namespace dsa {
+
+constexpr int kIndexerPage = 64;
+constexpr int kNumSMs = 148;
+
+// Lightning Indexer on CUDA cores (fp32 q/k; any heads <= 64, dim <= 128, dim % 4 == 0).
+cudaError_t launch_indexer_generic(const void* q, const float* q_scale, const float* w, int heads,
+                                   int dim, const CacheView& k, const BatchView& bv, float* logits,
+                                   long long ld, int* check, cudaStream_t st);
+
+// Lightning Indexer on tcgen05 tensor cores (fp8 e4m3 q/k, 64 heads x 128 dims).
+cudaError_t launch_indexer_fp8_tc(const void* q, const float* q_scale, const float* w,
+                                  const CacheView& k, const BatchView& bv, float* logits,
+                                  long long ld, int* check, cudaStream_t st);
+
+// Per-row top-k by radix select.
+cudaError_t launch_topk(const float* logits, long long ld, const BatchView& bv, int k, int* idx,
+                        int* check, cudaStream_t st);
+
+// Sparse MLA on CUDA cores (fp32 q/KV).  nsplit > 1 writes partials (o/l, lse) to
+// o_part [T][nsplit][heads][d_v] / lse_part [T][nsplit][heads] instead of out/lse.
+cudaError_t launch_mla_generic(const void* q, int heads, int d_qk, int d_v, float scale,
+                               const CacheView& kv, const BatchView& bv, const int* idx, int k,
+                               int nsplit, void* out, int out_dtype, float* lse, float* o_part,
+                               float* lse_part, int* check, cudaStream_t st);
+
+// Sparse MLA on tcgen05 tensor cores: bf16 q, bf16 or fp8 KV, 128 heads, 576 / 512.
+cudaError_t launch_mla_tc(const void* q, float scale, const CacheView& kv, const BatchView& bv,
+                          const int* idx, int k, int nsplit, void* out, float* lse, float* o_part,
+                          float* lse_part, int* check, cudaStream_t st);
+
+// Log-sum-exp merge of split partials into out (out_dtype) and lse.
+cudaError_t launch_mla_combine(const float* o_part, const float* lse_part, int total_q, int nsplit,
+                               int heads, int d_v, void* out, int out_dtype, float* lse,
+                               cudaStream_t st);
+
+}  // namespace dsa

@@ -1,0 +1,166 @@
+// mla_generic.cu -- sparse MLA on CUDA cores, and the log-sum-exp merge of split
+// partial results.
+//
+// For query row t and head h, over the selected positions s (idx[t][.], -1 skipped):
+//   z_s = softmax_scale * q[t,h,:] . (kv_s * kv_scale[s]),  p = softmax(z),
+//   o[t,h,:] = sum_s p_s * kv_s[0:d_v] * kv_scale[s],  lse = log sum_s exp(z_s)
+// (core attention over the top-k entries only: "SGLang Day-0 support for
+// DeepSeek-V3.2", section "DeepSeek Sparse Attention"; V is the first d_v columns
+// of the latent row).
+//
+// One warp owns one (query, head): it keeps q and its slice of o in registers,
+// walks the selected rows with an online softmax, and reduces each dot product
+// with shuffles.  With nsplit > 1 the selection list is cut into nsplit equal
+// chunks and each chunk writes a normalised partial (o/l, lse) for the merge.
+#include "kernels.h"
+
+namespace dsa {
+namespace {
+
+constexpr int kWarpsPerBlock = 4;
+constexpr int kMaxQK = 576;  // 18 per lane
+constexpr int kMaxV = 512;   // 16 per lane
+
+template <int QDT, int KVDT>
+__global__ void __launch_bounds__(32 * kWarpsPerBlock)
+mla_generic_kernel(const void* __restrict__ q, int heads, int d_qk, int d_v, float scale,
+                   CacheView kv, BatchView bv, const int* __restrict__ idx, int k, int nsplit,
+                   void* __restrict__ out, int out_dtype, float* __restrict__ lse,
+                   float* __restrict__ o_part, float* __restrict__ lse_part, int* check) {
+    const int t = blockIdx.x, split = blockIdx.z;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int h = blockIdx.y * kWarpsPerBlock + warp;
+    if (h >= heads) return;
+    const RowInfo ri = row_info(bv, t, check);
+
+    float qv[kMaxQK / 32];
+#pragma unroll
+    for (int j = 0; j < kMaxQK / 32; ++j) {
+        const int d = lane + 32 * j;
+        qv[j] = d < d_qk ? load_as_f32<QDT>(q, ((long long)t * heads + h) * d_qk + d) : 0.f;
+    }
+    float o[kMaxV / 32];
+#pragma unroll
+    for (int j = 0; j < kMaxV / 32; ++j) o[j] = 0.f;
+    float m = -INFINITY, l = 0.f;
+
+    const int chunk = (k + nsplit - 1) / nsplit;
+    const int i0 = split * chunk, i1 = min(k, i0 + chunk);
+    for (int i = i0; ri.ok && i < i1; ++i) {
+        const int s = __ldg(idx + (long long)t * k + i);
+        if (s < 0) continue;
+        if (s > ri.pos) {
+            if (lane == 0) report(check, kCheckBadIndex);
+            continue;
+        }
+        const long long r = cache_row(kv, ri.b, s, check);
+        if (r < 0) continue;
+        const float sc = kv.scale ? __ldg(kv.scale + r) : 1.0f;
+        float dot = 0.f;
+#pragma unroll
+        for (int j = 0; j < kMaxQK / 32; ++j) {
+            const int d = lane + 32 * j;
+            if (d < d_qk) dot = fmaf(qv[j], load_as_f32<KVDT>(kv.data, r * d_qk + d), dot);
+        }
+#pragma unroll
+        for (int off = 16; off; off >>= 1) dot += __shfl_xor_sync(0xffffffffu, dot, off);
+        const float z = dot * sc * scale;
+        const float m_new = fmaxf(m, z);
+        const float alpha = __expf(m - m_new);
+        const float p = __expf(z - m_new);
+        l = l * alpha + p;
+        const float ps = p * sc;
+#pragma unroll
+        for (int j = 0; j < kMaxV / 32; ++j) {
+            const int d = lane + 32 * j;
+            const float v = d < d_v ? load_as_f32<KVDT>(kv.data, r * d_qk + d) : 0.f;
+            o[j] = fmaf(o[j], alpha, ps * v);
+        }
+        m = m_new;
+    }
+    const float inv = l > 0.f ? 1.0f / l : 0.f;
+    const float lse_v = l > 0.f ? m + logf(l) : -INFINITY;
+    if (nsplit == 1) {
+        const long long base = ((long long)t * heads + h) * d_v;
+#pragma unroll
+        for (int j = 0; j < kMaxV / 32; ++j) {
+            const int d = lane + 32 * j;
+            if (d >= d_v) continue;
+            const float v = o[j] * inv;
+            if (out_dtype == kBF16) reinterpret_cast<__nv_bfloat16*>(out)[base + d] = __float2bfloat16_rn(v);
+            else reinterpret_cast<float*>(out)[base + d] = v;
+        }
+        if (lse && lane == 0) lse[(long long)t * heads + h] = lse_v;
+    } else {
+        const long long pbase = (((long long)t * nsplit + split) * heads + h);
+#pragma unroll
+        for (int j = 0; j < kMaxV / 32; ++j) {
+            const int d = lane + 32 * j;
+            if (d < d_v) o_part[pbase * d_v + d] = o[j] * inv;
+        }
+        if (lane == 0) lse_part[pbase] = lse_v;
+    }
+}
+
+// One CTA per (query, head): weights exp(lse_i - max) over the splits.
+__global__ void mla_combine_kernel(const float* __restrict__ o_part,
+                                   const float* __restrict__ lse_part, int nsplit, int heads,
+                                   int d_v, void* __restrict__ out, int out_dtype,
+                                   float* __restrict__ lse) {
+    const int t = blockIdx.x / heads, h = blockIdx.x % heads;
+    float mx = -INFINITY;
+    for (int i = 0; i < nsplit; ++i)
+        mx = fmaxf(mx, __ldg(lse_part + ((long long)t * nsplit + i) * heads + h));
+    float wsum = 0.f;
+    for (int i = 0; i < nsplit; ++i) {
+        const float li = __ldg(lse_part + ((long long)t * nsplit + i) * heads + h);
+        wsum += mx == -INFINITY ? 0.f : __expf(li - mx);
+    }
+    const float inv = wsum > 0.f ? 1.0f / wsum : 0.f;
+    for (int d = threadIdx.x; d < d_v; d += blockDim.x) {
+        float acc = 0.f;
+        for (int i = 0; i < nsplit; ++i) {
+            const long long pb = ((long long)t * nsplit + i) * heads + h;
+            const float li = __ldg(lse_part + pb);
+            if (li == -INFINITY) continue;
+            acc = fmaf(__expf(li - mx), __ldg(o_part + pb * d_v + d), acc);
+        }
+        const float v = acc * inv;
+        const long long ob = ((long long)t * heads + h) * d_v + d;
+        if (out_dtype == kBF16) reinterpret_cast<__nv_bfloat16*>(out)[ob] = __float2bfloat16_rn(v);
+        else reinterpret_cast<float*>(out)[ob] = v;
+    }
+    if (lse && threadIdx.x == 0)
+        lse[(long long)t * heads + h] = wsum > 0.f ? mx + logf(wsum) : -INFINITY;
+}
+
+}  // namespace
+
+cudaError_t launch_mla_generic(const void* q, int heads, int d_qk, int d_v, float scale,
+                               const CacheView& kv, const BatchView& bv, const int* idx, int k,
+                               int nsplit, void* out, int out_dtype, float* lse, float* o_part,
+                               float* lse_part, int* check, cudaStream_t st) {
+    dim3 grid(bv.total_q, (heads + kWarpsPerBlock - 1) / kWarpsPerBlock, nsplit);
+    dim3 block(32 * kWarpsPerBlock);
+    // fp32 q with fp32 KV, or bf16 q with bf16 / fp8 KV.
+    if (kv.dtype == kF32)
+        mla_generic_kernel<kF32, kF32><<<grid, block, 0, st>>>(q, heads, d_qk, d_v, scale, kv, bv,
+            idx, k, nsplit, out, out_dtype, lse, o_part, lse_part, check);
+    else if (kv.dtype == kBF16)
+        mla_generic_kernel<kBF16, kBF16><<<grid, block, 0, st>>>(q, heads, d_qk, d_v, scale, kv,
+            bv, idx, k, nsplit, out, out_dtype, lse, o_part, lse_part, check);
+    else
+        mla_generic_kernel<kBF16, kE4M3><<<grid, block, 0, st>>>(q, heads, d_qk, d_v, scale, kv,
+            bv, idx, k, nsplit, out, out_dtype, lse, o_part, lse_part, check);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_mla_combine(const float* o_part, const float* lse_part, int total_q, int nsplit,
+                               int heads, int d_v, void* out, int out_dtype, float* lse,
+                               cudaStream_t st) {
+    mla_combine_kernel<<<total_q * heads, 128, 0, st>>>(o_part, lse_part, nsplit, heads, d_v, out,
+                                                        out_dtype, lse);
+    return cudaGetLastError();
+}
+
+}  // namespace dsa

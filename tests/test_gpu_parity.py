@@ -1,0 +1,173 @@
+"""GPU parity of libdsa against the CPU oracle, through the C ABI.
+
+Each workload shape runs at full size in the launch configuration the benchmark
+uses; the oracle recomputes sampled query rows (all rows where it finishes in
+seconds).  Tolerances are stated in tests/_helpers.py.
+"""
+import math
+
+import numpy as np
+import pytest
+import torch
+
+import long_context_sparse_fp8_b200 as L
+from long_context_sparse_fp8_b200 import workloads as W
+
+import _helpers as H
+
+pytestmark = pytest.mark.gpu
+
+_CACHE = {}
+
+
+def _wl(key, spec_fn):
+    if key not in _CACHE:
+        _CACHE.clear()
+        torch.cuda.empty_cache()
+        _CACHE[key] = W.make(spec_fn(), device="cuda")
+    return _CACHE[key]
+
+
+def _pipeline(wl, rows, decode=False, atol=H.MLA_ATOL_BF16):
+    assert L.dsa_device_check() == 0
+    logits = H.run_indexer(wl)
+    idx = H.run_topk(wl, logits)
+    out, lse = H.run_mla(wl, idx, decode=decode)
+    torch.cuda.synchronize()
+    assert L.dsa_device_check() == 0
+    pos = H.positions(wl)[rows]
+    rows_t = torch.from_numpy(rows).cuda()
+    g_logits = logits[rows_t].cpu().numpy()
+    o_logits = H.oracle_logits(wl, rows)
+    H.check_logits(g_logits, o_logits, pos)
+    g_idx = idx[rows_t].cpu().numpy()
+    H.check_topk(g_idx, g_logits, o_logits, pos, wl.spec.topk)
+    o_ref, l_ref = H.oracle_mla(wl, g_idx, rows)
+    H.check_mla(out[rows_t].float().cpu().numpy(), lse[rows_t].cpu().numpy(), o_ref, l_ref, atol)
+    return logits, idx, out, lse
+
+
+def test_tiny_prefill_all_rows():
+    wl = W.make(W.tiny_prefill(), device="cuda")
+    _pipeline(wl, np.arange(wl.spec.total_q), atol=H.MLA_ATOL_F32)
+
+
+def test_decode_b32_ctx8192():
+    wl = _wl("c2", W.decode_b32_8k)
+    _pipeline(wl, H.sample_rows(32, 12, seed=2), decode=True)
+
+
+def test_fused_decode_matches_separate_calls():
+    wl = _wl("c2", W.decode_b32_8k)
+    s = wl.spec
+    batch, kc, kv = H.lib_args(wl)
+    logits = H.run_indexer(wl)
+    idx = H.run_topk(wl, logits)
+    out, lse = H.run_mla(wl, idx, decode=True)
+    n = L.dsa_decode_workspace_size(batch, s.topk, s.heads, s.d_v)
+    ws = torch.empty(n, dtype=torch.uint8, device="cuda")
+    out2 = torch.empty_like(out)
+    lse2 = torch.empty_like(lse)
+    idx2 = torch.empty_like(idx)
+    L.dsa_decode(wl.q_idx, None, wl.w, kc, s.topk, wl.q, kv, batch, s.d_v, s.softmax_scale, out2,
+                 lse2, idx2, ws)
+    torch.cuda.synchronize()
+    assert L.dsa_device_check() == 0
+    assert torch.equal(torch.sort(idx, 1).values, torch.sort(idx2, 1).values)
+    assert torch.equal(out, out2)
+    assert torch.equal(lse, lse2)
+
+
+def test_prefill_32k_heavy_hitters():
+    wl = _wl("c3", W.prefill_32k)
+    _pipeline(wl, H.sample_rows(wl.spec.total_q, 12, seed=3))
+
+
+def test_decode_b64_paged_fp8_kv():
+    wl = _wl("c4", W.decode_b64_128k)
+    _pipeline(wl, H.sample_rows(64, 6, seed=4), decode=True)
+
+
+@pytest.mark.parametrize("chunk", [0, 15])
+def test_chunked_prefill_128k(chunk):
+    wl = _wl(f"c5-{chunk}", lambda: W.chunked_prefill_128k(chunk))
+    _pipeline(wl, H.sample_rows(wl.spec.total_q, 6, seed=5 + chunk))
+
+
+@pytest.mark.parametrize("kv_fp8,permute", [(False, False), (True, True)])
+def test_ragged_batch_edge_cases(kv_fp8, permute):
+    """Lengths around page edges, L < k, a sequence with no queries, many queries."""
+    spec = W.Spec(name="ragged", seq_lens=[1, 63, 64, 65, 200, 2100, 3000, 2049],
+                  nq=[1, 5, 64, 2, 0, 7, 30, 3], topk=2048, kv_fp8=kv_fp8,
+                  permute_tables=permute, seed=77)
+    wl = W.make(spec, device="cuda")
+    _pipeline(wl, np.arange(spec.total_q))
+    _pipeline(wl, np.arange(spec.total_q), decode=True)
+
+
+def test_small_k_and_fp32_mla_split():
+    spec = W.tiny_prefill(seed=99)
+    spec.seq_lens, spec.nq, spec.topk = [300, 129], [40, 129], 16
+    wl = W.make(spec, device="cuda")
+    _pipeline(wl, np.arange(spec.total_q), atol=H.MLA_ATOL_F32)
+    _pipeline(wl, np.arange(spec.total_q), decode=True, atol=H.MLA_ATOL_F32)
+
+
+@pytest.mark.parametrize("n,k,kind", [(5000, 2048, "equal"), (5000, 2048, "three"),
+                                      (2049, 2048, "zeros"), (70000, 2048, "three"),
+                                      (70000, 2048, "normal"), (2048, 2048, "normal"),
+                                      (100000, 4096, "equal")])
+def test_topk_ties_and_long_rows(n, k, kind):
+    g = torch.Generator(device="cuda").manual_seed(n + k)
+    if kind == "equal":
+        row = torch.full((1, n), 1.5, device="cuda")
+    elif kind == "three":
+        row = torch.randint(0, 3, (1, n), generator=g, device="cuda").float()
+    elif kind == "zeros":  # +0.0 and -0.0 compare equal
+        row = torch.zeros(1, n, device="cuda")
+        row[0, ::2] = -0.0
+    else:
+        row = torch.randn(1, n, generator=g, device="cuda")
+    ld = (n + 3) // 4 * 4
+    logits = torch.full((1, ld), float("nan"), device="cuda")
+    logits[:, :n] = row
+    batch = L.Batch(torch.tensor([0, 1], dtype=torch.int32, device="cuda"),
+                    torch.tensor([n], dtype=torch.int32, device="cuda"), 1, n)
+    idx = torch.empty(1, k, dtype=torch.int32, device="cuda")
+    L.dsa_topk(logits, batch, k, idx)
+    got = idx.cpu().numpy()
+    H.check_topk(got, logits.cpu().numpy(), logits.cpu().numpy(), np.array([n - 1]), k)
+    if kind == "equal":
+        assert np.array_equal(np.sort(got[0]), np.arange(k))
+
+
+def test_device_check_reports_bad_index_and_page():
+    spec = W.Spec(name="chk", seq_lens=[300], nq=[4], topk=64, seed=5)
+    wl = W.make(spec, device="cuda")
+    assert L.dsa_device_check() == 0
+    logits = H.run_indexer(wl)
+    idx = H.run_topk(wl, logits)
+    torch.cuda.synchronize()
+    assert L.dsa_device_check() == 0
+    bad = idx.clone()
+    bad[0, 3] = 299  # row 0 sits at position 296
+    out, lse = H.run_mla(wl, bad)
+    assert L.dsa_device_check(reset=True) == 2  # DSA_CHECK_BAD_INDEX
+    assert torch.isfinite(out.float()).all()
+    assert L.dsa_device_check() == 0
+    wl.k_block_table[0, 2] = 10_000  # outside the page pool
+    H.run_indexer(wl)
+    assert L.dsa_device_check(reset=True) == 1  # DSA_CHECK_BAD_PAGE
+
+
+def test_empty_batch_is_a_no_op():
+    spec = W.Spec(name="empty", seq_lens=[10], nq=[0], topk=8, seed=1)
+    wl = W.make(spec, device="cuda")
+    batch, kc, kv = H.lib_args(wl)
+    logits = torch.full((1, 64), 3.0, device="cuda")
+    L.dsa_indexer_logits(wl.q_idx, None, wl.w, kc, batch, logits)
+    idx = torch.full((1, 8), 5, dtype=torch.int32, device="cuda")
+    L.dsa_topk(logits, batch, 8, idx)
+    torch.cuda.synchronize()
+    assert L.dsa_device_check() == 0
+    assert torch.all(logits == 3.0) and torch.all(idx == 5)
