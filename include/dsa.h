@@ -130,8 +130,8 @@ DSA_API dsa_status_t dsa_indexer_logits(const void* q, dsa_dtype_t q_dtype, cons
 
 /*
  * dsa_topk -- per-row top-k selection over logits[t][0..pos(t)].
- *   idx [T][k] int32 output: the selected positions (order unspecified when
- *   pos+1 > k, ascending otherwise), then -1 padding.  1 <= k <= 65536.
+ *   idx [T][k] int32 output: the selected positions in ascending order, then
+ *   -1 padding.  1 <= k <= 65536.  The result is deterministic.
  *   Ties at the k-th score keep the lowest positions; -0.0 equals +0.0.
  *   Logits must not be NaN.
  */

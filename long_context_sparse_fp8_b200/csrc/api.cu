@@ -133,6 +133,8 @@ dsa_status_t indexer_validate(const void* q, dsa_dtype_t q_dtype, const float* q
 cudaError_t indexer_launch(const void* q, const float* q_scale, const float* w, int heads, int dim,
                            const CacheView& kc, const BatchView& bv, float* logits, long long ld,
                            int* check, cudaStream_t st) {
+    if (kc.dtype == kE4M3)  // validated: 64 heads x 128 dims
+        return launch_indexer_fp8_tc(q, q_scale, w, kc, bv, logits, ld, check, st);
     return launch_indexer_generic(q, q_scale, w, heads, dim, kc, bv, logits, ld, check, st);
 }
 

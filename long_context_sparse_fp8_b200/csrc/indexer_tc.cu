@@ -1,0 +1,364 @@
+// indexer_tc.cu -- Lightning Indexer scores on sm_100a tensor cores (fp8 e4m3).
+//
+// I[t,s] = k_scale[s] * q_scale[t] * sum_j w[t,j] * ReLU(q[t,j,:] . k[s,:]),  s <= pos(t)
+// The indexer is the light FP8 scorer of "SGLang Day-0 support for
+// DeepSeek-V3.2", section "DeepSeek Sparse Attention"; its key & key_scale cache
+// uses page size 64 (same section); the deployment guide (m.nxbn.cn, section 3.1)
+// runs it in FP8.
+//
+// Mapping.  One tile = 128 keys (two 64-token pages) x (r query rows x 64 heads):
+//   D[key, (row, head)] = K_tile (128 x 128 fp8, K-major) . Q_rows^T (64r x 128 fp8)
+// is one tcgen05 kind::f8f6f4 MMA chain (M = 128, N = 64r, K = 4 x 32) into a TMEM
+// accumulator.  Each epilogue thread owns one key (one TMEM lane) and reduces its
+// row: sum_h w[row,h] * max(D, 0), then applies the key's and the query's scale.
+//
+// Roles (192 threads): warp 0 issues TMA loads (pages through the block table into
+// a 4-stage ring of 128-byte-swizzled tiles), warp 1 allocates TMEM and issues the
+// MMAs (double-buffered accumulators), warps 2-5 drain TMEM and write the logits.
+//
+// Grid: x = groups of G consecutive query rows (G = 1 for decode-like batches,
+// 4 otherwise; a group that spans sequences is processed as per-sequence runs),
+// y = chunks of the key tiles, so that short batches still cover all SMs.
+#include <cudaTypedefs.h>
+
+#include <mutex>
+
+#include "kernels.h"
+#include "sm100.cuh"
+
+namespace dsa {
+namespace {
+
+using namespace sm100;
+
+constexpr int kHeads = 64;
+constexpr int kDim = 128;
+constexpr int kTileKeys = 128;
+constexpr int kStages = 4;
+constexpr int kTileBytes = kTileKeys * kDim;       // 16 KB
+constexpr int kRowBytes = kHeads * kDim;            // one query row: 8 KB
+constexpr int kThreads = 192;
+
+struct Params {
+    const float* w;
+    const float* q_scale;
+    const float* k_scale;
+    const int* table;
+    long long num_pages;
+    int bt_stride;
+    BatchView bv;
+    float* logits;
+    long long ld;
+    int G;          // query rows per CTA
+    int C;          // key tiles per chunk
+    int* check;
+};
+
+struct Run {        // a run of query rows of one sequence
+    int b, t0, r, pos_lo, j0, j1;
+};
+
+// The r-th per-sequence run of the CTA's row group, restricted to its key chunk.
+// Returns false when there is no such run.
+__device__ __forceinline__ bool get_run(const Params& p, int k, Run* out) {
+    const int t_begin = blockIdx.x * p.G;
+    const int t_end = min(p.bv.total_q, t_begin + p.G);
+    int t = t_begin;
+    for (int i = 0; t < t_end; ++i) {
+        const int b = find_seq(p.bv.cu_q, p.bv.num_seqs, t);
+        const int q0 = __ldg(p.bv.cu_q + b), q1 = __ldg(p.bv.cu_q + b + 1);
+        const int L = __ldg(p.bv.seq_lens + b);
+        const int r = min(t_end, q1) - t;
+        if (i == k) {
+            out->b = b;
+            out->t0 = t;
+            out->r = r;
+            out->pos_lo = L - (q1 - q0) + (t - q0);
+            const bool ok = (q1 - q0) <= L && L <= p.bv.max_seq_len && out->pos_lo >= 0;
+            const int pos_hi = out->pos_lo + r - 1;
+            const int tiles = ok ? (pos_hi + kTileKeys) / kTileKeys : 0;
+            out->j0 = blockIdx.y * p.C;
+            out->j1 = min(tiles, out->j0 + p.C);
+            return true;
+        }
+        t += r;
+    }
+    return false;
+}
+
+__device__ __forceinline__ int page_of(const Params& p, int b, int s, int* bad) {
+    const int page = __ldg(p.table + (long long)b * p.bt_stride + s / 64);
+    if (page < 0 || (long long)page >= p.num_pages) {
+        *bad = 1;
+        return 0;
+    }
+    *bad = 0;
+    return page;
+}
+
+__global__ void __launch_bounds__(kThreads, 2)
+indexer_fp8_tc_kernel(const __grid_constant__ CUtensorMap tm_k,
+                      const __grid_constant__ CUtensorMap tm_q, Params p) {
+    extern __shared__ uint8_t smem_raw[];
+    // 1024-byte aligned carve-up: stages | Q (G rows) | w | barriers
+    uint8_t* base = reinterpret_cast<uint8_t*>(
+        (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    uint8_t* a_tiles = base;
+    uint8_t* q_tile = a_tiles + kStages * kTileBytes;
+    float* w_s = reinterpret_cast<float*>(q_tile + p.G * kRowBytes);   // [G][64]
+    uint64_t* bars = reinterpret_cast<uint64_t*>(w_s + p.G * kHeads);
+    uint64_t* full = bars;                    // [kStages] TMA -> MMA
+    uint64_t* empty = bars + kStages;         // [kStages] MMA -> TMA
+    uint64_t* tfull = bars + 2 * kStages;     // [2] MMA -> epilogue
+    uint64_t* tempty = tfull + 2;             // [2] epilogue -> MMA
+    uint64_t* qfull = tempty + 2;             // Q rows landed
+    uint64_t* qempty = qfull + 1;             // MMAs of a run done with Q
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(qempty + 1);
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int ncols_buf = p.G * kHeads;                     // accumulator columns per buffer
+    const uint32_t tmem_cols = ncols_buf * 2 <= 128 ? 128u : (ncols_buf * 2 <= 256 ? 256u : 512u);
+
+    if (threadIdx.x == 0) {
+        for (int i = 0; i < kStages; ++i) {
+            mbar_init(&full[i], 1);
+            mbar_init(&empty[i], 1);
+        }
+        for (int i = 0; i < 2; ++i) {
+            mbar_init(&tfull[i], 1);
+            mbar_init(&tempty[i], 4);   // one arrive per epilogue warp
+        }
+        mbar_init(qfull, 1);
+        mbar_init(qempty, 1);
+        fence_barrier_init();
+    }
+    if (warp == 1) {
+        tmem_alloc(tmem_slot, tmem_cols);
+        tmem_relinquish();
+    }
+    if (warp == 0 && lane == 0) {
+        prefetch_tmap(&tm_k);
+        prefetch_tmap(&tm_q);
+    }
+    {   // head weights of the CTA's rows, loaded once (no per-run barrier needed)
+        const int t_begin = blockIdx.x * p.G;
+        const int nrow = min(p.G, p.bv.total_q - t_begin);
+        for (int i = threadIdx.x; i < nrow * kHeads; i += kThreads)
+            w_s[i] = __ldg(p.w + (long long)t_begin * kHeads + i);
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem_base = *tmem_slot;
+
+    if (warp == 0) {
+        // ------------------------------------------------------------ TMA producer
+        if (elect_one()) {
+            int it = 0, runs_issued = 0;
+            bool alive = true;
+            Run run;
+            for (int k = 0; alive && get_run(p, k, &run); ++k) {
+                if (run.j0 >= run.j1) continue;
+                if (runs_issued > 0) {
+                    // the previous run's MMAs must be done reading Q
+                    if (!mbar_wait(qempty, (runs_issued - 1) & 1, p.check)) { alive = false; break; }
+                }
+                ++runs_issued;
+                mbar_arrive_expect_tx(qfull, p.G * kRowBytes);
+                tma_load_2d(q_tile, &tm_q, 0, run.t0 * kHeads, qfull);
+                const int pos_hi = run.pos_lo + run.r - 1;
+                for (int j = run.j0; j < run.j1; ++j, ++it) {
+                    const int stage = it % kStages;
+                    const uint32_t ph = (it / kStages) & 1;
+                    if (!mbar_wait(&empty[stage], ph ^ 1, p.check)) { alive = false; break; }
+                    int bad0, bad1 = 0;
+                    const int p0 = page_of(p, run.b, j * kTileKeys, &bad0);
+                    const bool two = j * kTileKeys + 64 <= pos_hi;
+                    const int p1 = two ? page_of(p, run.b, j * kTileKeys + 64, &bad1) : 0;
+                    if (bad0 | bad1) report(p.check, kCheckBadPage);
+                    mbar_arrive_expect_tx(&full[stage], two ? kTileBytes : kTileBytes / 2);
+                    uint8_t* dst = a_tiles + stage * kTileBytes;
+                    tma_load_2d(dst, &tm_k, 0, p0 * 64, &full[stage]);
+                    if (two) tma_load_2d(dst + kTileBytes / 2, &tm_k, 0, p1 * 64, &full[stage]);
+                }
+            }
+            // drain: every issued stage has been consumed (its empty phase completed)
+            const int n = it < kStages ? it : kStages;
+            for (int i = 0; i < n && alive; ++i) {
+                const int itx = it - 1 - i;
+                if (!mbar_wait(&empty[itx % kStages], (itx / kStages) & 1, p.check)) break;
+            }
+        }
+    } else if (warp == 1) {
+        // ------------------------------------------------------------ MMA issuer
+        if (elect_one()) {
+            int it = 0, runs_done = 0;
+            bool alive = true;
+            Run run;
+            const uint32_t q_addr = smem_u32(q_tile);
+            for (int k = 0; alive && get_run(p, k, &run); ++k) {
+                if (run.j0 >= run.j1) continue;
+                if (!mbar_wait(qfull, runs_done & 1, p.check)) { alive = false; break; }
+                tc_fence_after();
+                const uint32_t idesc = instr_desc(0, 0, 0, 0, run.r * kHeads, kTileKeys);
+                const uint64_t bdesc = smem_desc(q_addr, 16, 1024, kLayoutSw128);
+                for (int j = run.j0; j < run.j1; ++j, ++it) {
+                    const int stage = it % kStages;
+                    const int buf = it & 1;
+                    if (!mbar_wait(&tempty[buf], ((it >> 1) & 1) ^ 1, p.check)) { alive = false; break; }
+                    if (!mbar_wait(&full[stage], (it / kStages) & 1, p.check)) { alive = false; break; }
+                    tc_fence_after();
+                    const uint32_t d = tmem_base + buf * ncols_buf;
+                    const uint64_t adesc =
+                        smem_desc(smem_u32(a_tiles + stage * kTileBytes), 16, 1024, kLayoutSw128);
+#pragma unroll
+                    for (int kk = 0; kk < kDim / 32; ++kk)   // 32 fp8 = 32 bytes per K step
+                        mma_f8(d, adesc + 2 * kk, bdesc + 2 * kk, idesc, kk > 0 ? 1u : 0u);
+                    mma_commit(&empty[stage]);
+                    mma_commit(&tfull[buf]);
+                }
+                ++runs_done;
+                // free Q for a following run (not after the last one)
+                Run nxt;
+                bool more = false;
+                for (int k2 = k + 1; get_run(p, k2, &nxt); ++k2)
+                    if (nxt.j0 < nxt.j1) { more = true; break; }
+                if (more) mma_commit(qempty);
+            }
+        }
+    } else {
+        // ------------------------------------------------------------ epilogue
+        const int quarter = warp & 3;                 // TMEM lane quarter this warp may access
+        const int row = quarter * 32 + lane;          // key row within the tile
+        int it = 0;
+        bool alive = true;
+        Run run;
+        for (int k = 0; alive && get_run(p, k, &run); ++k) {
+            if (run.j0 >= run.j1) continue;
+            const float* w_run = w_s + (run.t0 - blockIdx.x * p.G) * kHeads;
+            float qs[4];
+#pragma unroll
+            for (int i = 0; i < 4; ++i)
+                qs[i] = (i < run.r && p.q_scale) ? __ldg(p.q_scale + run.t0 + i) : 1.0f;
+            const int pos_hi = run.pos_lo + run.r - 1;
+            for (int j = run.j0; j < run.j1; ++j, ++it) {
+                const int buf = it & 1;
+                const int s = j * kTileKeys + row;
+                float ks = 0.f;
+                int bad = 1;
+                if (s <= pos_hi) {
+                    const int page = page_of(p, run.b, s, &bad);
+                    ks = p.k_scale ? __ldg(p.k_scale + (long long)page * 64 + (s & 63)) : 1.0f;
+                }
+                if (!mbar_wait(&tfull[buf], (it >> 1) & 1, p.check)) { alive = false; break; }
+                tc_fence_after();
+                float res[4] = {0.f, 0.f, 0.f, 0.f};
+                const uint32_t tbase = tmem_base + ((uint32_t)(quarter * 32) << 16) + buf * ncols_buf;
+#pragma unroll
+                for (int qi = 0; qi < 4; ++qi) {
+                    if (qi >= run.r) break;
+                    uint32_t v0[32], v1[32];
+                    tmem_ld32(tbase + qi * kHeads, v0);
+                    tmem_ld32(tbase + qi * kHeads + 32, v1);
+                    tmem_ld_wait();
+                    const float4* w4 = reinterpret_cast<const float4*>(w_run + qi * kHeads);
+                    float acc = 0.f;
+#pragma unroll
+                    for (int h4 = 0; h4 < 8; ++h4) {
+                        const float4 wa = w4[h4];
+                        acc = fmaf(wa.x, fmaxf(__uint_as_float(v0[4 * h4 + 0]), 0.f), acc);
+                        acc = fmaf(wa.y, fmaxf(__uint_as_float(v0[4 * h4 + 1]), 0.f), acc);
+                        acc = fmaf(wa.z, fmaxf(__uint_as_float(v0[4 * h4 + 2]), 0.f), acc);
+                        acc = fmaf(wa.w, fmaxf(__uint_as_float(v0[4 * h4 + 3]), 0.f), acc);
+                    }
+#pragma unroll
+                    for (int h4 = 0; h4 < 8; ++h4) {
+                        const float4 wa = w4[8 + h4];
+                        acc = fmaf(wa.x, fmaxf(__uint_as_float(v1[4 * h4 + 0]), 0.f), acc);
+                        acc = fmaf(wa.y, fmaxf(__uint_as_float(v1[4 * h4 + 1]), 0.f), acc);
+                        acc = fmaf(wa.z, fmaxf(__uint_as_float(v1[4 * h4 + 2]), 0.f), acc);
+                        acc = fmaf(wa.w, fmaxf(__uint_as_float(v1[4 * h4 + 3]), 0.f), acc);
+                    }
+                    res[qi] = acc;
+                }
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&tempty[buf]);
+#pragma unroll
+                for (int qi = 0; qi < 4; ++qi) {
+                    if (qi >= run.r) break;
+                    const int pos = run.pos_lo + qi;
+                    float* dst = p.logits + (long long)(run.t0 + qi) * p.ld + s;
+                    if (s <= pos) *dst = bad ? -INFINITY : res[qi] * ks * qs[qi];
+                    else if (s < p.ld) *dst = -INFINITY;
+                }
+            }
+        }
+    }
+
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    if (warp == 1) tmem_dealloc(tmem_base, tmem_cols);
+}
+
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+    static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void* ptr = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) ==
+                cudaSuccess && q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(ptr);
+    });
+    return fn;
+}
+
+// 2-D byte matrix [rows][128] with a 128 x box_rows box, 128-byte swizzle.
+cudaError_t make_map(CUtensorMap* m, const void* base, unsigned long long rows, uint32_t box_rows) {
+    auto fn = encode_fn();
+    if (!fn) return cudaErrorNotSupported;
+    cuuint64_t dims[2] = {128, rows};
+    cuuint64_t strides[1] = {128};
+    cuuint32_t box[2] = {128, box_rows};
+    cuuint32_t estr[2] = {1, 1};
+    CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(base), dims, strides,
+                    box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                    CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS ? cudaSuccess : cudaErrorInvalidValue;
+}
+
+}  // namespace
+
+cudaError_t launch_indexer_fp8_tc(const void* q, const float* q_scale, const float* w,
+                                  const CacheView& k, const BatchView& bv, float* logits,
+                                  long long ld, int* check, cudaStream_t st) {
+    const int T = bv.total_q;
+    const int G = T <= 2 * bv.num_seqs ? 1 : 4;
+    const int groups = (T + G - 1) / G;
+    const int tiles_max = (bv.max_seq_len + kTileKeys - 1) / kTileKeys;
+    const int target = 4 * kNumSMs;
+    int chunks = groups >= target / 2 ? 1 : (target + groups - 1) / groups;
+    if (chunks > tiles_max) chunks = tiles_max;
+    const int C = (tiles_max + chunks - 1) / chunks;
+    chunks = (tiles_max + C - 1) / C;
+
+    CUtensorMap tm_k, tm_q;
+    cudaError_t e = make_map(&tm_k, k.data, (unsigned long long)k.num_pages * 64, 64);
+    if (e != cudaSuccess) return e;
+    e = make_map(&tm_q, q, (unsigned long long)T * kHeads, G * kHeads);
+    if (e != cudaSuccess) return e;
+
+    Params p{w, q_scale, k.scale, k.table, k.num_pages, k.bt_stride, bv, logits, ld, G, C, check};
+    const size_t smem = 1024 + kStages * kTileBytes + (size_t)G * kRowBytes +
+                        (size_t)G * kHeads * sizeof(float) + 16 * sizeof(uint64_t) + 16;
+    e = cudaFuncSetAttribute(indexer_fp8_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             (int)smem);
+    if (e != cudaSuccess) return e;
+    dim3 grid(groups, chunks);
+    indexer_fp8_tc_kernel<<<grid, kThreads, smem, st>>>(tm_k, tm_q, p);
+    return cudaGetLastError();
+}
+
+}  // namespace dsa

@@ -7,8 +7,8 @@
 // Method: exact radix select on order-preserving 32-bit keys.  One 1024-thread CTA
 // owns one row.  Three histogram passes (11 + 11 + 10 bits, shared-memory
 // atomics) pin down the exact k-th largest key T and how many keys equal to T
-// are still needed; a final pass emits every key > T and the lowest-position
-// keys == T.  Rows of up to kSmemKeys candidates are staged once in shared
+// are still needed; a final two-pass emission writes every key > T and the
+// lowest-position keys == T in ascending position order (deterministic output).  Rows of up to kSmemKeys candidates are staged once in shared
 // memory; longer rows are re-read from global memory (L2) on each pass.
 #include "kernels.h"
 
@@ -63,24 +63,13 @@ struct Row {
     }
 };
 
-// Appends `idx` for the lanes with `take` set, warp-aggregated, at out[*counter++].
-__device__ __forceinline__ void warp_append(bool take, int idx, int* counter, int* out) {
-    const unsigned m = __ballot_sync(0xffffffffu, take);
-    if (!m) return;
-    const int lane = threadIdx.x & 31;
-    int base = 0;
-    if (lane == __ffs(m) - 1) base = atomicAdd(counter, __popc(m));
-    base = __shfl_sync(0xffffffffu, base, __ffs(m) - 1);
-    if (take) out[base + __popc(m & ((1u << lane) - 1u))] = idx;
-}
-
 __global__ void __launch_bounds__(kThreads)
 topk_kernel(const float* __restrict__ logits, long long ld, BatchView bv, int k,
             int* __restrict__ idx, int* check, int smem_keys) {
     extern __shared__ uint32_t skeys[];
     __shared__ int hist[2048];
     __shared__ int warp_sums[kWarps + 1];
-    __shared__ int s_bin, s_above, s_count;
+    __shared__ int s_bin, s_above;
 
     const int t = blockIdx.x, tid = threadIdx.x;
     int* out = idx + (long long)t * k;
@@ -105,7 +94,6 @@ topk_kernel(const float* __restrict__ logits, long long ld, BatchView bv, int k,
     // ---- radix select: find the exact k-th largest key -------------------------
     uint32_t prefix = 0u, pmask = 0u;
     int remaining = k;   // how many of the keys matching `prefix` still have to be taken
-    int eq_total = 0;
     const int shifts[3] = {21, 10, 0};
     const int nbits[3] = {11, 11, 10};
 #pragma unroll 1
@@ -143,36 +131,50 @@ topk_kernel(const float* __restrict__ logits, long long ld, BatchView bv, int k,
         remaining -= s_above;
         prefix |= (uint32_t)bin << shift;
         pmask |= (uint32_t)(nb - 1) << shift;
-        eq_total = hist[bin];
         __syncthreads();
     }
     const uint32_t T = prefix;          // the k-th largest key
     const int need_eq = remaining;      // keys == T to take (>= 1)
-    const int gt_count = k - need_eq;   // keys > T (all taken)
 
-    // ---- emit ----------------------------------------------------------------
-    if (tid == 0) s_count = 0;
-    __syncthreads();
-    const bool all_eq = eq_total == need_eq;
-    const int iters = (n + kThreads - 1) / kThreads;
-    for (int it = 0; it < iters; ++it) {
-        const int i = it * kThreads + tid;
-        const uint32_t key = i < n ? row(i) : 0u;
-        const bool take = i < n && (key > T || (all_eq && key == T));
-        warp_append(take, i, &s_count, out);
+    // ---- emit, deterministic and in position order --------------------------
+    // Warp w owns the contiguous segment [w*seg, (w+1)*seg).  Pass A counts its
+    // keys > T and == T; a block scan turns the counts into offsets; pass B
+    // writes every key > T and the first need_eq keys == T (lowest positions).
+    const int lane = tid & 31, warp = tid >> 5;
+    const int seg = ((n + kWarps - 1) / kWarps + 31) & ~31;
+    const int w0 = min(n, warp * seg), w1 = min(n, w0 + seg);
+    int c_gt = 0, c_eq = 0;
+    for (int i0 = w0; i0 < w1; i0 += 32) {
+        const int i = i0 + lane;
+        const uint32_t key = i < w1 ? row(i) : 0u;
+        c_gt += __popc(__ballot_sync(0xffffffffu, i < w1 && key > T));
+        c_eq += __popc(__ballot_sync(0xffffffffu, i < w1 && key == T));
     }
-    if (!all_eq) {
-        // Ties at the threshold: the need_eq lowest positions with key == T, in
-        // position order, after the gt_count keys above T.
-        int base = 0;
-        for (int c0 = 0; c0 < n && base < need_eq; c0 += kThreads) {
-            const int i = c0 + tid;
-            const int flag = (i < n && row(i) == T) ? 1 : 0;
-            int total;
-            const int rank = block_excl_scan(flag, warp_sums, &total);
-            if (flag && base + rank < need_eq) out[gt_count + base + rank] = i;
-            base += total;
-        }
+    __shared__ int s_gt[kWarps], s_eq[kWarps];
+    if (lane == 0) {
+        s_gt[warp] = c_gt;
+        s_eq[warp] = c_eq;
+    }
+    __syncthreads();
+    int gt_before = 0, eq_before = 0;
+    for (int v = 0; v < warp; ++v) {
+        gt_before += s_gt[v];
+        eq_before += s_eq[v];
+    }
+    int taken = gt_before + min(eq_before, need_eq);   // output slot of the next taken key
+    int eq_seen = eq_before;
+    for (int i0 = w0; i0 < w1; i0 += 32) {
+        const int i = i0 + lane;
+        const uint32_t key = i < w1 ? row(i) : 0u;
+        const bool gt = i < w1 && key > T;
+        const bool eq = i < w1 && key == T;
+        const unsigned meq = __ballot_sync(0xffffffffu, eq);
+        const int eq_rank = eq_seen + __popc(meq & ((1u << lane) - 1u));
+        const bool take = gt || (eq && eq_rank < need_eq);
+        const unsigned mt = __ballot_sync(0xffffffffu, take);
+        if (take) out[taken + __popc(mt & ((1u << lane) - 1u))] = i;
+        taken += __popc(mt);
+        eq_seen += __popc(meq);
     }
 }
 

@@ -73,7 +73,7 @@ def test_fused_decode_matches_separate_calls():
                  lse2, idx2, ws)
     torch.cuda.synchronize()
     assert L.dsa_device_check() == 0
-    assert torch.equal(torch.sort(idx, 1).values, torch.sort(idx2, 1).values)
+    assert torch.equal(idx, idx2)          # top-k output is deterministic
     assert torch.equal(out, out2)
     assert torch.equal(lse, lse2)
 
