@@ -148,7 +148,8 @@ DSA_API dsa_status_t dsa_topk(const float* logits, int64_t ld_logits, const dsa_
  *            (natural log; -inf and o = 0 for a row with no valid index)
  * Kernels: BF16 q with BF16 or FP8 (per-token scale) KV, heads = 128,
  *          d_qk = 576, d_v = 512, out BF16 (tcgen05 tensor cores);
- *          F32 q/KV with heads <= 16, d_qk <= 576, d_v <= 512 (CUDA cores).
+ *          F32 q/KV with heads <= 16, d_qk <= 576, d_v <= 512, d_v % 4 == 0
+ *          (CUDA cores).
  */
 DSA_API dsa_status_t dsa_sparse_mla_prefill(const void* q, dsa_dtype_t q_dtype, int32_t heads,
                                             int32_t d_qk, int32_t d_v, float softmax_scale,

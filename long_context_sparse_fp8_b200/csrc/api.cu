@@ -174,8 +174,9 @@ dsa_status_t mla_check(const void* q, dsa_dtype_t q_dtype, int heads, int d_qk, 
     if (!valid_dtype(q_dtype) || !valid_dtype(out_dtype))
         return fail(DSA_ERR_INVALID_ARGUMENT, "q_dtype / out_dtype is not a dsa_dtype_t");
     if (q_dtype == DSA_F32 && plan->kv.dtype == kF32) {
-        if (d_qk > 576 || d_v > 512 || heads > 16)
-            return fail(DSA_ERR_UNSUPPORTED, "fp32 sparse MLA supports heads <= 16, d_qk <= 576, d_v <= 512");
+        if (d_qk > 576 || d_v > 512 || heads > 16 || d_v % 4 != 0)
+            return fail(DSA_ERR_UNSUPPORTED, "fp32 sparse MLA supports heads <= 16, d_qk <= 576, "
+                        "d_v <= 512 with d_v %% 4 == 0");
         if (out_dtype != DSA_F32 && out_dtype != DSA_BF16)
             return fail(DSA_ERR_UNSUPPORTED, "fp32 sparse MLA writes fp32 or bf16 output");
         plan->kind = MlaKind::kGenericF32;
@@ -195,6 +196,9 @@ cudaError_t mla_launch(const MlaPlan& plan, const void* q, int heads, int d_qk, 
                        float scale, const BatchView& bv, const int* idx, int k, int nsplit,
                        void* out, int out_dtype, float* lse, float* o_part, float* lse_part,
                        int* check, cudaStream_t st) {
+    if (plan.kind == MlaKind::kTensorCore)
+        return launch_mla_tc(q, scale, plan.kv, bv, idx, k, nsplit, out, lse, o_part, lse_part,
+                             check, st);
     return launch_mla_generic(q, heads, d_qk, d_v, scale, plan.kv, bv, idx, k, nsplit, out,
                               out_dtype, lse, o_part, lse_part, check, st);
 }

@@ -54,13 +54,13 @@ struct Params {
     int* check;
 };
 
-struct Run {        // a run of query rows of one sequence
+struct Run {        // a run of query rows of one sequence (j0 == j1: nothing to do)
     int b, t0, r, pos_lo, j0, j1;
 };
 
 // The r-th per-sequence run of the CTA's row group, restricted to its key chunk.
 // Returns false when there is no such run.
-__device__ __forceinline__ bool get_run(const Params& p, int k, Run* out) {
+__device__ __forceinline__ bool get_run(const Params& p, int k, Run* out, bool skip) {
     const int t_begin = blockIdx.x * p.G;
     const int t_end = min(p.bv.total_q, t_begin + p.G);
     int t = t_begin;
@@ -78,7 +78,7 @@ __device__ __forceinline__ bool get_run(const Params& p, int k, Run* out) {
             const int pos_hi = out->pos_lo + r - 1;
             const int tiles = ok ? (pos_hi + kTileKeys) / kTileKeys : 0;
             out->j0 = blockIdx.y * p.C;
-            out->j1 = min(tiles, out->j0 + p.C);
+            out->j1 = skip ? out->j0 : min(tiles, out->j0 + p.C);
             return true;
         }
         t += r;
@@ -119,7 +119,9 @@ indexer_fp8_tc_kernel(const __grid_constant__ CUtensorMap tm_k,
     const int ncols_buf = p.G * kHeads;                     // accumulator columns per buffer
     const uint32_t tmem_cols = ncols_buf * 2 <= 128 ? 128u : (ncols_buf * 2 <= 256 ? 256u : 512u);
 
+    __shared__ int s_skip;
     if (threadIdx.x == 0) {
+        s_skip = timed_out_before(p.check) ? 1 : 0;
         for (int i = 0; i < kStages; ++i) {
             mbar_init(&full[i], 1);
             mbar_init(&empty[i], 1);
@@ -150,6 +152,7 @@ indexer_fp8_tc_kernel(const __grid_constant__ CUtensorMap tm_k,
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem_base = *tmem_slot;
+    const bool skip = s_skip != 0;   // an earlier CTA timed out: do no work
 
     if (warp == 0) {
         // ------------------------------------------------------------ TMA producer
@@ -157,7 +160,7 @@ indexer_fp8_tc_kernel(const __grid_constant__ CUtensorMap tm_k,
             int it = 0, runs_issued = 0;
             bool alive = true;
             Run run;
-            for (int k = 0; alive && get_run(p, k, &run); ++k) {
+            for (int k = 0; alive && get_run(p, k, &run, skip); ++k) {
                 if (run.j0 >= run.j1) continue;
                 if (runs_issued > 0) {
                     // the previous run's MMAs must be done reading Q
@@ -196,7 +199,7 @@ indexer_fp8_tc_kernel(const __grid_constant__ CUtensorMap tm_k,
             bool alive = true;
             Run run;
             const uint32_t q_addr = smem_u32(q_tile);
-            for (int k = 0; alive && get_run(p, k, &run); ++k) {
+            for (int k = 0; alive && get_run(p, k, &run, skip); ++k) {
                 if (run.j0 >= run.j1) continue;
                 if (!mbar_wait(qfull, runs_done & 1, p.check)) { alive = false; break; }
                 tc_fence_after();
@@ -221,7 +224,7 @@ indexer_fp8_tc_kernel(const __grid_constant__ CUtensorMap tm_k,
                 // free Q for a following run (not after the last one)
                 Run nxt;
                 bool more = false;
-                for (int k2 = k + 1; get_run(p, k2, &nxt); ++k2)
+                for (int k2 = k + 1; get_run(p, k2, &nxt, skip); ++k2)
                     if (nxt.j0 < nxt.j1) { more = true; break; }
                 if (more) mma_commit(qempty);
             }
@@ -233,7 +236,7 @@ indexer_fp8_tc_kernel(const __grid_constant__ CUtensorMap tm_k,
         int it = 0;
         bool alive = true;
         Run run;
-        for (int k = 0; alive && get_run(p, k, &run); ++k) {
+        for (int k = 0; alive && get_run(p, k, &run, skip); ++k) {
             if (run.j0 >= run.j1) continue;
             const float* w_run = w_s + (run.t0 - blockIdx.x * p.G) * kHeads;
             float qs[4];

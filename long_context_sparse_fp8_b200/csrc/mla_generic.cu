@@ -1,5 +1,5 @@
-// mla_generic.cu -- sparse MLA on CUDA cores, and the log-sum-exp merge of split
-// partial results.
+// mla_generic.cu -- sparse MLA on CUDA cores for fp32 inputs, and the log-sum-exp
+// merge of split partial results (shared with the tensor-core kernel).
 //
 // For query row t and head h, over the selected positions s (idx[t][.], -1 skipped):
 //   z_s = softmax_scale * q[t,h,:] . (kv_s * kv_scale[s]),  p = softmax(z),
@@ -102,35 +102,45 @@ mla_generic_kernel(const void* __restrict__ q, int heads, int d_qk, int d_v, flo
     }
 }
 
-// One CTA per (query, head): weights exp(lse_i - max) over the splits.
-__global__ void mla_combine_kernel(const float* __restrict__ o_part,
-                                   const float* __restrict__ lse_part, int nsplit, int heads,
-                                   int d_v, void* __restrict__ out, int out_dtype,
-                                   float* __restrict__ lse) {
-    const int t = blockIdx.x / heads, h = blockIdx.x % heads;
+// Merge of split partials: o = sum_i exp(lse_i - lse) o_i with lse = log sum_i exp(lse_i).
+// One thread per 4 output values of one (query, head); a block covers 2 heads x 512.
+__global__ void __launch_bounds__(256)
+mla_combine_kernel(const float* __restrict__ o_part, const float* __restrict__ lse_part,
+                   int nsplit, int heads, int d_v, void* __restrict__ out, int out_dtype,
+                   float* __restrict__ lse) {
+    const int t = blockIdx.x;
+    const int per_head = d_v / 4;                       // threads per head
+    const int h = blockIdx.y * (blockDim.x / per_head) + threadIdx.x / per_head;
+    const int d4 = threadIdx.x % per_head;
+    if (h >= heads) return;
     float mx = -INFINITY;
     for (int i = 0; i < nsplit; ++i)
         mx = fmaxf(mx, __ldg(lse_part + ((long long)t * nsplit + i) * heads + h));
     float wsum = 0.f;
+    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
     for (int i = 0; i < nsplit; ++i) {
-        const float li = __ldg(lse_part + ((long long)t * nsplit + i) * heads + h);
-        wsum += mx == -INFINITY ? 0.f : __expf(li - mx);
+        const long long pb = ((long long)t * nsplit + i) * heads + h;
+        const float li = __ldg(lse_part + pb);
+        if (li == -INFINITY) continue;
+        const float wgt = __expf(li - mx);
+        wsum += wgt;
+        const float4 v = __ldg(reinterpret_cast<const float4*>(o_part + pb * d_v) + d4);
+        acc.x = fmaf(wgt, v.x, acc.x);
+        acc.y = fmaf(wgt, v.y, acc.y);
+        acc.z = fmaf(wgt, v.z, acc.z);
+        acc.w = fmaf(wgt, v.w, acc.w);
     }
     const float inv = wsum > 0.f ? 1.0f / wsum : 0.f;
-    for (int d = threadIdx.x; d < d_v; d += blockDim.x) {
-        float acc = 0.f;
-        for (int i = 0; i < nsplit; ++i) {
-            const long long pb = ((long long)t * nsplit + i) * heads + h;
-            const float li = __ldg(lse_part + pb);
-            if (li == -INFINITY) continue;
-            acc = fmaf(__expf(li - mx), __ldg(o_part + pb * d_v + d), acc);
-        }
-        const float v = acc * inv;
-        const long long ob = ((long long)t * heads + h) * d_v + d;
-        if (out_dtype == kBF16) reinterpret_cast<__nv_bfloat16*>(out)[ob] = __float2bfloat16_rn(v);
-        else reinterpret_cast<float*>(out)[ob] = v;
+    const long long ob = ((long long)t * heads + h) * d_v + 4 * d4;
+    if (out_dtype == kBF16) {
+        __nv_bfloat162* o2 = reinterpret_cast<__nv_bfloat162*>(reinterpret_cast<__nv_bfloat16*>(out) + ob);
+        o2[0] = __floats2bfloat162_rn(acc.x * inv, acc.y * inv);
+        o2[1] = __floats2bfloat162_rn(acc.z * inv, acc.w * inv);
+    } else {
+        *reinterpret_cast<float4*>(reinterpret_cast<float*>(out) + ob) =
+            make_float4(acc.x * inv, acc.y * inv, acc.z * inv, acc.w * inv);
     }
-    if (lse && threadIdx.x == 0)
+    if (lse && d4 == 0)
         lse[(long long)t * heads + h] = wsum > 0.f ? mx + logf(wsum) : -INFINITY;
 }
 
@@ -142,24 +152,21 @@ cudaError_t launch_mla_generic(const void* q, int heads, int d_qk, int d_v, floa
                                float* lse_part, int* check, cudaStream_t st) {
     dim3 grid(bv.total_q, (heads + kWarpsPerBlock - 1) / kWarpsPerBlock, nsplit);
     dim3 block(32 * kWarpsPerBlock);
-    // fp32 q with fp32 KV, or bf16 q with bf16 / fp8 KV.
-    if (kv.dtype == kF32)
-        mla_generic_kernel<kF32, kF32><<<grid, block, 0, st>>>(q, heads, d_qk, d_v, scale, kv, bv,
-            idx, k, nsplit, out, out_dtype, lse, o_part, lse_part, check);
-    else if (kv.dtype == kBF16)
-        mla_generic_kernel<kBF16, kBF16><<<grid, block, 0, st>>>(q, heads, d_qk, d_v, scale, kv,
-            bv, idx, k, nsplit, out, out_dtype, lse, o_part, lse_part, check);
-    else
-        mla_generic_kernel<kBF16, kE4M3><<<grid, block, 0, st>>>(q, heads, d_qk, d_v, scale, kv,
-            bv, idx, k, nsplit, out, out_dtype, lse, o_part, lse_part, check);
+    // fp32 q with fp32 KV (bf16 / fp8 KV runs on the tensor-core kernel)
+    mla_generic_kernel<kF32, kF32><<<grid, block, 0, st>>>(q, heads, d_qk, d_v, scale, kv, bv,
+        idx, k, nsplit, out, out_dtype, lse, o_part, lse_part, check);
     return cudaGetLastError();
 }
 
 cudaError_t launch_mla_combine(const float* o_part, const float* lse_part, int total_q, int nsplit,
                                int heads, int d_v, void* out, int out_dtype, float* lse,
                                cudaStream_t st) {
-    mla_combine_kernel<<<total_q * heads, 128, 0, st>>>(o_part, lse_part, nsplit, heads, d_v, out,
-                                                        out_dtype, lse);
+    // d_v % 4 == 0 and d_v <= 512 (validated by the callers)
+    const int per_head = d_v / 4;
+    const int heads_per_block = per_head >= 256 ? 1 : 256 / per_head;
+    dim3 grid(total_q, (heads + heads_per_block - 1) / heads_per_block);
+    mla_combine_kernel<<<grid, per_head * heads_per_block, 0, st>>>(o_part, lse_part, nsplit,
+                                                                   heads, d_v, out, out_dtype, lse);
     return cudaGetLastError();
 }
 

@@ -43,9 +43,16 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
     return ok != 0;
 }
 
-// Waits for phase `parity` of `bar` to complete, giving up after ~2 s of SM clock:
-// then records DSA_CHECK_TIMEOUT and returns false, so the caller can unwind.
-constexpr long long kWaitLimitCycles = 4000000000LL;
+// Waits for phase `parity` of `bar` to complete, giving up after ~0.1 s of SM
+// clock (legitimate waits last microseconds): then records DSA_CHECK_TIMEOUT and
+// returns false, so the caller can unwind.
+constexpr long long kWaitLimitCycles = 200000000LL;
+
+// True once any CTA has recorded a timeout: later CTAs of the launch skip their
+// work instead of waiting out the limit again.
+__device__ __forceinline__ bool timed_out_before(const int* check) {
+    return check && *reinterpret_cast<const volatile int*>(check) == kCheckTimeout;
+}
 
 __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, int* check) {
     if (mbar_try_wait(bar, parity)) return true;
@@ -57,6 +64,61 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, int* c
         }
     }
     return true;
+}
+
+// Same wait with cluster-scope acquire: for data a peer CTA wrote into this
+// CTA's shared memory before arriving remotely.
+__device__ __forceinline__ bool mbar_try_wait_cluster(uint64_t* bar, uint32_t parity) {
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok) : "r"(smem_u32(bar)), "r"(parity) : "memory");
+    return ok != 0;
+}
+
+__device__ __forceinline__ bool mbar_wait_cluster(uint64_t* bar, uint32_t parity, int* check) {
+    if (mbar_try_wait_cluster(bar, parity)) return true;
+    const long long t0 = clock64();
+    while (!mbar_try_wait_cluster(bar, parity)) {
+        if (clock64() - t0 > kWaitLimitCycles) {
+            report(check, kCheckTimeout);
+            return false;
+        }
+    }
+    return true;
+}
+
+// ---------------------------------------------------------------- clusters
+__device__ __forceinline__ uint32_t cluster_ctarank() {
+    uint32_t r;
+    asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+    return r;
+}
+
+// Address of the same shared-memory location in CTA `rank` of the cluster.
+__device__ __forceinline__ uint32_t mapa(uint32_t saddr, uint32_t rank) {
+    uint32_t r;
+    asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(saddr), "r"(rank));
+    return r;
+}
+
+__device__ __forceinline__ void st_cluster_v4(uint32_t caddr, float a, float b, float c, float d) {
+    asm volatile("st.shared::cluster.v4.f32 [%0], {%1, %2, %3, %4};"
+                 ::"r"(caddr), "f"(a), "f"(b), "f"(c), "f"(d) : "memory");
+}
+
+// Arrive on a peer CTA's mbarrier, releasing this thread's prior writes cluster-wide.
+__device__ __forceinline__ void mbar_arrive_remote(uint32_t caddr) {
+    asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];"
+                 ::"r"(caddr) : "memory");
+}
+
+// All threads of both CTAs (must be executed convergently by every warp).
+__device__ __forceinline__ void cluster_sync() {
+    asm volatile("barrier.cluster.arrive.release.aligned;\n\t"
+                 "barrier.cluster.wait.acquire.aligned;" ::: "memory");
 }
 
 __device__ __forceinline__ void fence_proxy_async_smem() {
