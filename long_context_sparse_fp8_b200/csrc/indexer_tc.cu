@@ -253,7 +253,7 @@ indexer_fp8_tc_kernel(const __grid_constant__ CUtensorMap tm_k,
                     const int page = page_of(p, run.b, s, &bad);
                     ks = p.k_scale ? __ldg(p.k_scale + (long long)page * 64 + (s & 63)) : 1.0f;
                 }
-                if (!mbar_wait(&tfull[buf], (it >> 1) & 1, p.check)) { alive = false; break; }
+                if (!mbar_wait_warp(&tfull[buf], (it >> 1) & 1, p.check)) { alive = false; break; }
                 tc_fence_after();
                 float res[4] = {0.f, 0.f, 0.f, 0.f};
                 const uint32_t tbase = tmem_base + ((uint32_t)(quarter * 32) << 16) + buf * ncols_buf;

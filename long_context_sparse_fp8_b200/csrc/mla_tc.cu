@@ -8,28 +8,31 @@
 // KV cache: "DeepSeek V3.2 usage guide", attention-kernel section; 128 heads,
 // 576 = 512 latent + 64 rope, V = the 512 latent columns).
 //
-// Why a CTA pair.  The fp32 output tile O (128 heads x 512) fills all 512 TMEM
-// columns of an SM, leaving no room for the score tile.  So a 2-CTA cluster works
-// on one (query, split): rank r owns V columns [256r, 256r+256) and the 288 dims
-// D_r = [256r, 256r+256) u [512+32r, 512+32r+32) of the QK contraction.  Each rank
-// gathers only D_r of every selected row (no byte is fetched twice), computes the
-// partial scores S_r = Q[:, D_r] . KV[:, D_r]^T on tcgen05, and the two partial
-// tiles are swapped through distributed shared memory.  Both ranks add them
-// (S_0 + S_1 == S_1 + S_0 bit for bit), so both run an identical online softmax,
-// write the same P tile, and accumulate O[:, 256r:256r+256] += P . V_r.
+// Why two CTAs per query.  The fp32 output tile O (128 heads x 512) would fill all
+// 512 TMEM columns of an SM, leaving no room for the scores.  So CTA v (v = 0, 1)
+// of a (query, split) owns V columns [256v, 256v+256): it computes the full score
+// tile S = Q . KV^T (K = 576) itself, runs the softmax, and accumulates its half of
+// O.  The two CTAs repeat the QK product (1.5x the unique tensor work) but never
+// talk to each other: exchanging partial score tiles through distributed shared
+// memory moves only ~8 bytes per cycle between a CTA pair, slower than recomputing.
 //
-// Roles (288 threads per CTA): warps 0-3 = softmax (thread = head = TMEM lane),
-// warps 4-7 = gather (2 threads per selected row, loads issued one tile ahead),
-// warp 8 = TMEM owner and MMA issuer.  The MMAs run on fp16 operands: e4m3 and
-// bf16 values convert to fp16 exactly (bf16 magnitudes above 65504 saturate), and
-// the probabilities P get 11 significant bits instead of bf16's 8.
-// Per 64-row tile: 18 MMAs (M=128, N=64, K=16) for S_r, 4 MMAs (M=128, N=256,
-// K=16) for P.V_r.  Online softmax in base 2 with lazy rescaling: O and l are only
-// rescaled when the running max grows by more than 2^8.
+// Roles (352 threads): warps 0-3 = softmax (thread = head = TMEM lane), warps 4-9 =
+// gather (3 threads per selected row), warp 10 = TMEM owner and MMA issuer.  The
+// gather is software-pipelined over tiles, per thread: the index of tile j+4, the
+// slot of tile j+3, an L2 bulk prefetch of the rows of tile j+2 and the register
+// loads of tile j+1 are all in flight while tile j is written to shared memory.  The MMAs run on fp16 operands: e4m3 and bf16 values
+// convert to fp16 exactly (bf16 magnitudes above 65504 saturate), and P keeps 11
+// significant bits.
 //
-// Shared memory (one CTA per SM): Q_r 72 KB, 2 KV stages x 36 KB, one exchange
-// buffer of 32 KB, 2 P buffers x 16 KB.  Tiles of 64 dims are 128-byte swizzled K-major; the
-// 32 rope dims of a rank use the no-swizzle core-matrix layout.
+// Tensor memory: O_v (256 columns), S (64), P (32 = 64 fp16) and query dims 0..319
+// (160 columns); dims 320..575 of the query sit in shared memory next to a 2-stage
+// ring of gathered 64-row tiles (72 KB each, 128-byte swizzled K-major regions of
+// 64 dims).  Per tile: 36 MMAs (M=128, N=64, K=16) for S -- A from TMEM or shared
+// memory -- and 4 MMAs (M=128, N=256, K=16) for P.V_v with A = P in TMEM.  Online
+// softmax in base 2 with lazy rescaling (O and l are rescaled only when the running
+// max grows by more than 2^8).
+#include <climits>
+
 #include "kernels.h"
 #include "sm100.cuh"
 
@@ -40,27 +43,31 @@ using namespace sm100;
 
 constexpr int kHeads = 128;
 constexpr int kTile = 64;
-constexpr int kThreads = 288;
+constexpr int kThreads = 352;
 constexpr int kGatherWarp0 = 4;
-constexpr int kMmaWarp = 8;
+constexpr int kGatherThreads = 192;    // 3 per row of a 64-row tile
+constexpr int kMmaWarp = 10;
 
-constexpr uint32_t kQBytes = 4 * 16384 + 8192;
-constexpr uint32_t kStageBytes = 4 * 8192 + 4096;
-constexpr uint32_t kXBytes = kHeads * kTile * 4;
-constexpr uint32_t kPBytes = kHeads * kTile * 2;
-constexpr uint32_t kOffQ = 0;
-constexpr uint32_t kOffKV = kOffQ + kQBytes;
-constexpr uint32_t kOffX = kOffKV + 2 * kStageBytes;
-constexpr uint32_t kOffP = kOffX + kXBytes;             // [2] P tiles
-constexpr uint32_t kOffFlag = kOffP + 2 * kPBytes;      // [2][64] validity bytes
-constexpr uint32_t kOffScale = kOffFlag + 128;          // [2][64] fp32 per-row kv scale
-constexpr uint32_t kOffBar = kOffScale + 512;
-constexpr uint32_t kSmemBytes = kOffBar + 16 * 8 + 16 + 1024;
+constexpr int kStages = 2;
+constexpr int kRegions = 9;                              // 64-dim regions of a 576-dim row
+constexpr uint32_t kQsRegions = 4;                       // query dims 320..575 in smem
+constexpr uint32_t kQsBytes = kQsRegions * 16384;        // 128 rows x 128 B per region
+constexpr uint32_t kStageBytes = kRegions * 8192;        // 64 rows x 128 B per region
+constexpr uint32_t kOffQs = 0;
+constexpr uint32_t kOffKV = kOffQs + kQsBytes;
+constexpr uint32_t kOffFlag = kOffKV + kStages * kStageBytes;   // [stage][64] validity bytes
+constexpr uint32_t kOffScale = kOffFlag + kStages * 64;         // [stage][64] fp32 kv scale
+constexpr uint32_t kOffBar = kOffScale + kStages * 256;
+constexpr uint32_t kNumBars = 12;
+constexpr uint32_t kSmemBytes = kOffBar + kNumBars * 8 + 16 + 1024;
 static_assert(kSmemBytes <= 232448, "shared memory budget");
 
 constexpr uint32_t kTmemCols = 512;
-constexpr uint32_t kColS = 0;      // two 64-column score buffers
-constexpr uint32_t kColO = 256;    // 256 output columns
+constexpr uint32_t kColO = 0;      // 256 output columns
+constexpr uint32_t kColS = 256;    // 64 score columns
+constexpr uint32_t kColP = 320;    // 32 columns = 64 fp16 probabilities
+constexpr uint32_t kColQ = 352;    // 160 columns = query dims 0..319 as fp16 pairs
+constexpr int kQtSteps = 20;       // K-steps of 16 dims with A in TMEM
 
 struct Params {
     const uint4* q;            // bf16 [T][128][576] as 16-byte chunks (72 per head)
@@ -86,20 +93,6 @@ struct Params {
 __device__ __forceinline__ uint32_t sw128(int r, int c) {
     return (uint32_t)(r * 128 + ((c ^ (r & 7)) << 4));
 }
-// Byte offset of 16-byte chunk c (0..3) of row r in a no-swizzle tile of 64-byte
-// rows: 8x16-byte core matrices, K-adjacent ones 128 B apart, 8-row groups 512 B.
-__device__ __forceinline__ uint32_t il64(int r, int c) {
-    return (uint32_t)((r >> 3) * 512 + c * 128 + ((r & 7) << 4));
-}
-// Rank-local bf16 chunk g (0..35) of a row: chunk index in the 72-chunk global row.
-__device__ __forceinline__ int global_chunk(int rank, int g) {
-    return g < 32 ? 32 * rank + g : 64 + 4 * rank + (g - 32);
-}
-// Shared-memory offset of local chunk g of `row` (region stride rs, rope region r4).
-__device__ __forceinline__ uint32_t local_off(int row, int g, uint32_t rs, uint32_t r4) {
-    return g < 32 ? (uint32_t)(g >> 3) * rs + sw128(row, g & 7) : r4 + il64(row, g - 32);
-}
-
 __device__ __forceinline__ uint4 ldg16(const void* p) {
     uint4 v;
     asm volatile("ld.global.nc.v4.u32 {%0, %1, %2, %3}, [%4];"
@@ -110,13 +103,6 @@ __device__ __forceinline__ uint4 ldg16(const void* p) {
 __device__ __forceinline__ void sts16(uint32_t saddr, uint4 v) {
     asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};"
                  ::"r"(saddr), "r"(v.x), "r"(v.y), "r"(v.z), "r"(v.w) : "memory");
-}
-
-__device__ __forceinline__ float4 lds16f(uint32_t saddr) {
-    float4 v;
-    asm volatile("ld.shared.v4.f32 {%0, %1, %2, %3}, [%4];"
-                 : "=f"(v.x), "=f"(v.y), "=f"(v.z), "=f"(v.w) : "r"(saddr));
-    return v;
 }
 
 // Two e4m3 codes (low byte first) -> two fp16 (exact: every e4m3 value is an fp16).
@@ -154,7 +140,7 @@ __device__ __forceinline__ uint32_t pack_bf16(float a, float b) {
 }
 
 template <bool kFp8>
-__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
+__global__ void __launch_bounds__(kThreads, 1)
 mla_tc_kernel(const Params p) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t* base = reinterpret_cast<uint8_t*>(
@@ -163,37 +149,33 @@ mla_tc_kernel(const Params p) {
     uint8_t* vflag = base + kOffFlag;
     float* colscale = reinterpret_cast<float*>(base + kOffScale);
     uint64_t* bars = reinterpret_cast<uint64_t*>(base + kOffBar);
-    uint64_t* kvfull = bars + 0;    // [2] gather -> MMA / softmax     (128 arrivals)
+    uint64_t* kvfull = bars + 0;    // [2] gather -> MMA / softmax     (192 arrivals)
     uint64_t* kvempty = bars + 2;   // [2] PV done -> gather           (commit)
-    uint64_t* sfull = bars + 4;     // [2] S_r ready -> softmax        (commit)
-    uint64_t* sempty = bars + 6;    // [2] S_r read -> MMA             (128)
-    uint64_t* xfull = bars + 8;     // peer's partial landed           (4 remote, one per warp)
-    uint64_t* xempty = bars + 9;    // peer consumed our partial       (4 remote)
-    uint64_t* pfull = bars + 10;    // [2] P (and any O rescale) ready (128)
-    uint64_t* pvdone = bars + 12;   // [2] PV of that P buffer done    (commit)
-    uint64_t* qfull = bars + 14;    // Q_r in place                    (128)
-    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 16);
+    uint64_t* sfull = bars + 4;     // scores ready                    (commit)
+    uint64_t* sempty = bars + 5;    // scores read                     (128)
+    uint64_t* pfull = bars + 6;     // P (and any O rescale) ready     (128)
+    uint64_t* pvdone = bars + 7;    // PV finished                     (commit)
+    uint64_t* qfull = bars + 8;     // query in TMEM + shared memory   (128)
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + kNumBars);
 
     const int warp = threadIdx.x >> 5;
-    const uint32_t rank = cluster_ctarank(), peer = rank ^ 1u;
+    const int vh = blockIdx.x & 1;                   // which half of the V columns
     const int cid = blockIdx.x >> 1;
     const int t = cid / p.nsplit, split = cid % p.nsplit;
     const RowInfo ri = row_info(p.bv, t, threadIdx.x == 0 ? p.check : nullptr);
     const int i0 = split * p.chunk, i1 = min(p.k, i0 + p.chunk);
     __shared__ int s_skip;
-    if (threadIdx.x == 0) s_skip = timed_out_before(p.check) ? 1 : 0;
 
     if (threadIdx.x == 0) {
-        for (int i = 0; i < 2; ++i) {
-            mbar_init(&kvfull[i], 128);
+        s_skip = timed_out_before(p.check) ? 1 : 0;
+        for (int i = 0; i < kStages; ++i) {
+            mbar_init(&kvfull[i], kGatherThreads);
             mbar_init(&kvempty[i], 1);
-            mbar_init(&sfull[i], 1);
-            mbar_init(&sempty[i], 128);
-            mbar_init(&pfull[i], 128);
-            mbar_init(&pvdone[i], 1);
         }
-        mbar_init(xfull, 4);
-        mbar_init(xempty, 4);
+        mbar_init(sfull, 1);
+        mbar_init(sempty, 128);
+        mbar_init(pfull, 128);
+        mbar_init(pvdone, 1);
         mbar_init(qfull, 128);
         fence_barrier_init();
     }
@@ -203,92 +185,111 @@ mla_tc_kernel(const Params p) {
     }
     tc_fence_before();
     __syncthreads();
-    cluster_sync();   // the peer's barriers exist before any remote arrive
     tc_fence_after();
     const uint32_t tmem = *tmem_slot;
     const int n_tiles = (ri.ok && i1 > i0 && !s_skip) ? (i1 - i0 + kTile - 1) / kTile : 0;
 
     if (warp >= kGatherWarp0 && warp < kMmaWarp) {
         // ============================================================ gather
-        const int gt = threadIdx.x - kGatherWarp0 * 32;     // 0..127
-        {   // Q_r: head gt, its 36 rank-local chunks, as fp16
-            const uint4* qrow = p.q + ((long long)t * kHeads + gt) * 72;
-#pragma unroll
-            for (int g0 = 0; g0 < 36; g0 += 18) {
-                uint4 qv[18];
-#pragma unroll
-                for (int g = 0; g < 18; ++g)
-                    qv[g] = ri.ok ? ldg16(qrow + global_chunk(rank, g0 + g)) : make_uint4(0, 0, 0, 0);
-#pragma unroll
-                for (int g = 0; g < 18; ++g)
-                    sts16(sb + kOffQ + local_off(gt, g0 + g, 16384, 65536), bf16x8_to_f16x8(qv[g]));
-            }
-            fence_proxy_async_smem();
-            mbar_arrive(qfull);
-        }
-        const int c = gt >> 1, half = gt & 1;      // selected row of the tile, which half
-        constexpr int kN = kFp8 ? 9 : 18;          // 16-byte global loads per thread per tile
-        uint4 v[kN];
-        bool valid = false;
-        float scale = 0.f;
-        auto load = [&](int j) {
+        const int gt = threadIdx.x - kGatherWarp0 * 32;     // 0..191
+        const int c = gt / 3, part = gt % 3;                // row of the tile, third of the row
+        constexpr int kN = kFp8 ? 12 : 24;                  // 16-byte loads per thread per tile
+        constexpr int kRowBytes = kFp8 ? 576 : 1152;
+        const long long seq_base = (long long)ri.b * p.st_stride;
+        // Per-thread pipeline state for its row c of upcoming tiles: no load result is
+        // consumed in the iteration that issues the load.
+        int idx5 = -1;                                  // index of tile j+5
+        int raw_s4 = -1;                                // slot-table entry of tile j+4 (unchecked)
+        long long slot1 = -1, slot2 = -1, slot3 = -1;   // checked slots of tiles j+1..j+3
+        auto fetch_idx = [&](int j) -> int {
             const int i = i0 + j * kTile + c;
-            const int s = i < i1 ? __ldg(p.idx + (long long)t * p.k + i) : -1;
-            valid = s >= 0 && s <= ri.pos;
-            if (s > ri.pos && half == 0) report(p.check, kCheckBadIndex);
-            long long slot = 0;
-            if (valid) {
-                slot = __ldg(p.slot_table + (long long)ri.b * p.st_stride + s);
-                if (slot < 0 || slot >= p.num_slots) {
-                    if (half == 0) report(p.check, kCheckBadPage);
-                    valid = false;
-                }
-            }
-            scale = (valid && kFp8 && p.kv_scale) ? __ldg(p.kv_scale + slot) : 1.0f;
-            if constexpr (kFp8) {
-                const uint8_t* row = p.kv + slot * 576;
-#pragma unroll
-                for (int u = 0; u < kN; ++u) {
-                    const int gg = half * 9 + u;
-                    const int off = gg < 16 ? 256 * (int)rank + 16 * gg : 512 + 32 * (int)rank + 16 * (gg - 16);
-                    v[u] = valid ? ldg16(row + off) : make_uint4(0, 0, 0, 0);
-                }
-            } else {
-                const uint4* row = reinterpret_cast<const uint4*>(p.kv + slot * 1152);
-#pragma unroll
-                for (int u = 0; u < kN; ++u)
-                    v[u] = valid ? ldg16(row + global_chunk(rank, half * 18 + u)) : make_uint4(0, 0, 0, 0);
-            }
+            return (j < n_tiles && i < i1) ? __ldg(p.idx + (long long)t * p.k + i) : -1;
         };
-        if (n_tiles > 0) load(0);
+        // Slot-table entry for index s, or a sentinel for a skipped entry / an index
+        // past the query position (table entries are checked separately).
+        constexpr int kSkip = INT_MIN, kPastPos = INT_MIN + 1;
+        auto fetch_slot = [&](int s) -> int {
+            if (s < 0) return kSkip;
+            if (s > ri.pos) return kPastPos;
+            return __ldg(p.slot_table + seq_base + s);
+        };
+        auto check_slot = [&](int raw) -> long long {   // -1 for skipped / bad entries
+            if (raw == kSkip) return -1;
+            if (raw == kPastPos || raw < 0 || (long long)raw >= p.num_slots) {
+                if (part == 0) report(p.check, raw == kPastPos ? kCheckBadIndex : kCheckBadPage);
+                return -1;
+            }
+            return raw;
+        };
+        auto prefetch_row = [&](long long sl) {
+            if (sl >= 0)
+                asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;"
+                             ::"l"(p.kv + sl * kRowBytes + part * kN * 16), "r"(kN * 16) : "memory");
+        };
+        uint4 v[kN];
+        float scale = 1.0f;
+        auto load_regs = [&](long long sl) {
+            const uint4* row = reinterpret_cast<const uint4*>(p.kv + (sl < 0 ? 0 : sl) * kRowBytes) + part * kN;
+#pragma unroll
+            for (int u = 0; u < kN; ++u) v[u] = sl >= 0 ? ldg16(row + u) : make_uint4(0, 0, 0, 0);
+            scale = (sl >= 0 && kFp8 && p.kv_scale) ? __ldg(p.kv_scale + sl) : 1.0f;
+        };
+        // prologue: tiles 0..4 in flight
+        long long slot0 = -1;
+        if (n_tiles > 0) {
+            const int x0 = fetch_idx(0), x1 = fetch_idx(1), x2 = fetch_idx(2), x3 = fetch_idx(3),
+                      x4 = fetch_idx(4);
+            idx5 = fetch_idx(5);
+            const int r0 = fetch_slot(x0), r1 = fetch_slot(x1), r2 = fetch_slot(x2),
+                      r3 = fetch_slot(x3);
+            raw_s4 = fetch_slot(x4);
+            slot0 = check_slot(r0);
+            slot1 = check_slot(r1);
+            slot2 = check_slot(r2);
+            slot3 = check_slot(r3);
+            prefetch_row(slot1);
+            load_regs(slot0);
+        }
+        long long cur = slot0;                          // slot of the tile held in v
         for (int j = 0; j < n_tiles; ++j) {
-            const int stage = j & 1;
-            if (!mbar_wait(&kvempty[stage], ((j >> 1) & 1) ^ 1, p.check)) break;
+            const int stage = j % kStages;
+            if (!mbar_wait_warp(&kvempty[stage], ((j / kStages) & 1) ^ 1, p.check)) break;
             const uint32_t st = sb + kOffKV + stage * kStageBytes;
             if constexpr (kFp8) {
 #pragma unroll
                 for (int u = 0; u < kN; ++u) {
-                    const int gg = half * 9 + u;
+                    const int g = 2 * (part * kN + u);      // first of the two fp16 chunks
                     const uint4 a = v[u];
                     const uint4 lo = make_uint4(e4m3x2_to_f16x2(a.x & 0xFFFF), e4m3x2_to_f16x2(a.x >> 16),
                                                 e4m3x2_to_f16x2(a.y & 0xFFFF), e4m3x2_to_f16x2(a.y >> 16));
                     const uint4 hi = make_uint4(e4m3x2_to_f16x2(a.z & 0xFFFF), e4m3x2_to_f16x2(a.z >> 16),
                                                 e4m3x2_to_f16x2(a.w & 0xFFFF), e4m3x2_to_f16x2(a.w >> 16));
-                    sts16(st + local_off(c, 2 * gg, 8192, 32768), lo);
-                    sts16(st + local_off(c, 2 * gg + 1, 8192, 32768), hi);
+                    sts16(st + (g >> 3) * 8192 + sw128(c, g & 7), lo);
+                    sts16(st + ((g + 1) >> 3) * 8192 + sw128(c, (g + 1) & 7), hi);
                 }
             } else {
 #pragma unroll
-                for (int u = 0; u < kN; ++u)
-                    sts16(st + local_off(c, half * 18 + u, 8192, 32768), bf16x8_to_f16x8(v[u]));
+                for (int u = 0; u < kN; ++u) {
+                    const int g = part * kN + u;
+                    sts16(st + (g >> 3) * 8192 + sw128(c, g & 7), bf16x8_to_f16x8(v[u]));
+                }
             }
-            if (half == 0) {
-                vflag[stage * 64 + c] = valid ? 1 : 0;
+            if (part == 0) {
+                vflag[stage * 64 + c] = cur >= 0 ? 1 : 0;
                 colscale[stage * 64 + c] = scale;
             }
             fence_proxy_async_smem();
             mbar_arrive(&kvfull[stage]);
-            if (j + 1 < n_tiles) load(j + 1);
+            // advance the pipeline by one tile
+            if (j + 1 < n_tiles) load_regs(slot1);
+            prefetch_row(slot2);
+            const long long s4 = check_slot(raw_s4);   // loaded one iteration ago
+            raw_s4 = fetch_slot(idx5);                  // index loaded one iteration ago
+            idx5 = fetch_idx(j + 6);
+            cur = slot1;
+            slot1 = slot2;
+            slot2 = slot3;
+            slot3 = s4;
         }
     } else if (warp == kMmaWarp) {
         // ============================================================ MMA issuer
@@ -297,133 +298,148 @@ mla_tc_kernel(const Params p) {
             tc_fence_after();
             const uint32_t idesc_qk = instr_desc(0, 0, 0, 0, kTile, kHeads);   // fp16 x fp16
             const uint32_t idesc_pv = instr_desc(0, 0, 0, 1, 256, kHeads);
-            const uint32_t qa = sb + kOffQ;
-            const uint32_t pa = sb + kOffP;
+            const uint32_t qs = sb + kOffQs;
             for (int j = 0; alive && j <= n_tiles; ++j) {
                 if (j < n_tiles) {
-                    const int stage = j & 1, buf = j & 1;
-                    if (!mbar_wait(&kvfull[stage], (j >> 1) & 1, p.check)) break;
-                    if (!mbar_wait(&sempty[buf], ((j >> 1) & 1) ^ 1, p.check)) break;
+                    const int stage = j % kStages;
+                    if (!mbar_wait(&kvfull[stage], (j / kStages) & 1, p.check)) break;
+                    if (j >= 1 && !mbar_wait(sempty, (j - 1) & 1, p.check)) break;
                     tc_fence_after();
                     const uint32_t kva = sb + kOffKV + stage * kStageBytes;
-                    const uint32_t d = tmem + kColS + buf * kTile;
-                    uint32_t acc = 0;
 #pragma unroll
-                    for (int reg = 0; reg < 4; ++reg) {
-#pragma unroll
-                        for (int kk = 0; kk < 4; ++kk) {
-                            mma_f16(d, smem_desc(qa + reg * 16384 + kk * 32, 16, 1024, kLayoutSw128),
-                                    smem_desc(kva + reg * 8192 + kk * 32, 16, 1024, kLayoutSw128),
-                                    idesc_qk, acc);
-                            acc = 1;
-                        }
+                    for (int s = 0; s < 36; ++s) {
+                        const uint64_t bdesc =
+                            smem_desc(kva + (s >> 2) * 8192 + (s & 3) * 32, 16, 1024, kLayoutSw128);
+                        if (s < kQtSteps)
+                            mma_f16_ts(tmem + kColS, tmem + kColQ + 8 * s, bdesc, idesc_qk, s > 0 ? 1u : 0u);
+                        else
+                            mma_f16(tmem + kColS,
+                                    smem_desc(qs + ((s - kQtSteps) >> 2) * 16384 + (s & 3) * 32, 16, 1024,
+                                              kLayoutSw128),
+                                    bdesc, idesc_qk, 1u);
                     }
-#pragma unroll
-                    for (int kk = 0; kk < 2; ++kk)
-                        mma_f16(d, smem_desc(qa + 65536 + kk * 256, 128, 512, kLayoutNone),
-                                smem_desc(kva + 32768 + kk * 256, 128, 512, kLayoutNone), idesc_qk, 1);
-                    mma_commit(&sfull[buf]);
+                    mma_commit(sfull);
                 }
                 if (j >= 1) {
-                    const int jj = j - 1, stage = jj & 1;
-                    if (!mbar_wait(&pfull[jj & 1], (jj >> 1) & 1, p.check)) break;
+                    const int jj = j - 1, stage = jj % kStages;
+                    if (!mbar_wait(pfull, jj & 1, p.check)) break;
                     tc_fence_after();
-                    const uint32_t kva = sb + kOffKV + stage * kStageBytes;
-                    const uint32_t pb = pa + (jj & 1) * kPBytes;
+                    const uint32_t va = sb + kOffKV + stage * kStageBytes + vh * 4 * 8192;
 #pragma unroll
                     for (int kk = 0; kk < 4; ++kk)
-                        mma_f16(tmem + kColO, smem_desc(pb + kk * 32, 16, 1024, kLayoutSw128),
-                                smem_desc(kva + kk * 2048, 8192, 1024, kLayoutSw128), idesc_pv,
-                                (jj > 0 || kk > 0) ? 1u : 0u);
+                        mma_f16_ts(tmem + kColO, tmem + kColP + 8 * kk,
+                                   smem_desc(va + kk * 2048, 8192, 1024, kLayoutSw128), idesc_pv,
+                                   (jj > 0 || kk > 0) ? 1u : 0u);
                     mma_commit(&kvempty[stage]);
-                    mma_commit(&pvdone[jj & 1]);
+                    mma_commit(pvdone);
                 }
             }
         }
     } else {
         // ============================================================ softmax
         const int h = threadIdx.x;                       // head == TMEM lane
-        const int lane = threadIdx.x & 31;
         const uint32_t lane_base = tmem + ((uint32_t)(warp * 32) << 16);
-        const uint32_t xa = sb + kOffX;
-        const uint32_t peer_x = mapa(xa, peer);
-        const uint32_t peer_xfull = mapa(smem_u32(xfull), peer);   // the peer's own barriers
-        const uint32_t peer_xempty = mapa(smem_u32(xempty), peer);
+        {   // query row h: dims 0..319 into TMEM as fp16 pairs, 320..575 into smem
+            const uint4* qrow = p.q + ((long long)t * kHeads + h) * 72;
+            if (ri.ok) asm volatile("cp.async.bulk.prefetch.L2.global [%0], 1152;" ::"l"(qrow) : "memory");
+#pragma unroll
+            for (int g0 = 0; g0 < 72; g0 += 24) {
+                uint4 qv[24];
+#pragma unroll
+                for (int g = 0; g < 24; ++g) qv[g] = ri.ok ? ldg16(qrow + g0 + g) : make_uint4(0, 0, 0, 0);
+#pragma unroll
+                for (int g = 0; g < 24; g += 2) {
+                    const int gg = g0 + g;
+                    const uint4 a = bf16x8_to_f16x8(qv[g]), b = bf16x8_to_f16x8(qv[g + 1]);
+                    if (gg < 40) {
+                        tmem_st8(lane_base + kColQ + 4 * gg, a.x, a.y, a.z, a.w, b.x, b.y, b.z, b.w);
+                    } else {
+                        const int c0 = gg - 40;              // chunk index within dims 320..575
+                        sts16(sb + kOffQs + (c0 >> 3) * 16384 + sw128(h, c0 & 7), a);
+                        sts16(sb + kOffQs + ((c0 + 1) >> 3) * 16384 + sw128(h, (c0 + 1) & 7), b);
+                    }
+                }
+            }
+            tmem_st_wait();
+            fence_proxy_async_smem();
+            tc_fence_before();
+            mbar_arrive(qfull);
+        }
         float m_run = -INFINITY, l_run = 0.f;
         bool alive = true;
         for (int j = 0; alive && j < n_tiles; ++j) {
-            const int buf = j & 1, u = j >> 1;
-            // ---- this rank's partial scores
-            if (!mbar_wait(&sfull[buf], u & 1, p.check)) { alive = false; break; }
-            tc_fence_after();
-            uint32_t sr[64];
-            {
-                uint32_t a[32], b[32];
-                tmem_ld32(lane_base + kColS + buf * kTile, a);
-                tmem_ld32(lane_base + kColS + buf * kTile + 32, b);
+            const int stage = j % kStages;
+            float x[64];
+            {   // ---- scores of tile j
+                if (!mbar_wait_warp(sfull, j & 1, p.check)) { alive = false; break; }
+                tc_fence_after();
+                uint32_t a[32], c[32];
+                tmem_ld32(lane_base + kColS, a);
+                tmem_ld32(lane_base + kColS + 32, c);
                 tmem_ld_wait();
+                tc_fence_before();
+                mbar_arrive(sempty);                       // the next QK may overwrite S
 #pragma unroll
                 for (int i = 0; i < 32; ++i) {
-                    sr[i] = a[i];
-                    sr[32 + i] = b[i];
+                    x[i] = __uint_as_float(a[i]);
+                    x[32 + i] = __uint_as_float(c[i]);
                 }
             }
-            tc_fence_before();
-            mbar_arrive(&sempty[buf]);
-            // ---- swap partial tiles with the peer rank (one exchange buffer each)
-            if (j >= 1 && !mbar_wait_cluster(xempty, (j - 1) & 1, p.check)) { alive = false; break; }
-            const uint32_t xrow = (uint32_t)h * 256;
-#pragma unroll
-            for (int c4 = 0; c4 < 16; ++c4)
-                st_cluster_v4(peer_x + xrow + ((c4 ^ (h & 7)) << 4), __uint_as_float(sr[4 * c4]),
-                              __uint_as_float(sr[4 * c4 + 1]), __uint_as_float(sr[4 * c4 + 2]),
-                              __uint_as_float(sr[4 * c4 + 3]));
-            __syncwarp();
-            if (lane == 0) mbar_arrive_remote(peer_xfull);
-            if (!mbar_wait_cluster(xfull, j & 1, p.check)) { alive = false; break; }
-            float x[64];
-#pragma unroll
-            for (int c4 = 0; c4 < 16; ++c4) {
-                const float4 o = lds16f(xa + xrow + ((c4 ^ (h & 7)) << 4));
-                x[4 * c4 + 0] = __uint_as_float(sr[4 * c4 + 0]) + o.x;
-                x[4 * c4 + 1] = __uint_as_float(sr[4 * c4 + 1]) + o.y;
-                x[4 * c4 + 2] = __uint_as_float(sr[4 * c4 + 2]) + o.z;
-                x[4 * c4 + 3] = __uint_as_float(sr[4 * c4 + 3]) + o.w;
-            }
-            __syncwarp();
-            if (lane == 0) mbar_arrive_remote(peer_xempty);
             // ---- online softmax (base 2)
-            if (!mbar_wait(&kvfull[buf], u & 1, p.check)) { alive = false; break; }
-            const uint8_t* fl = vflag + buf * 64;
-            const float* cs = colscale + buf * 64;
-            float m_tile = -INFINITY;
+            if (!mbar_wait_warp(&kvfull[stage], (j / kStages) & 1, p.check)) { alive = false; break; }
+            const float* cs = colscale + stage * 64;
+            {   // invalid entries (skipped or bad indices) score -inf
+                const uint4* f4 = reinterpret_cast<const uint4*>(vflag + stage * 64);
+                uint4 w[4];
+                bool all = true;
 #pragma unroll
-            for (int i = 0; i < 64; ++i) {
-                const float sc = kFp8 ? p.sc_log2 * cs[i] : p.sc_log2;
-                x[i] = fl[i] ? x[i] * sc : -INFINITY;
-                m_tile = fmaxf(m_tile, x[i]);
+                for (int q = 0; q < 4; ++q) {
+                    w[q] = f4[q];
+                    all = all && w[q].x == 0x01010101u && w[q].y == 0x01010101u &&
+                          w[q].z == 0x01010101u && w[q].w == 0x01010101u;
+                }
+                if (!all) {
+#pragma unroll
+                    for (int q = 0; q < 4; ++q) {
+                        const uint32_t ws[4] = {w[q].x, w[q].y, w[q].z, w[q].w};
+#pragma unroll
+                        for (int b = 0; b < 16; ++b)
+                            if (!((ws[b >> 2] >> (8 * (b & 3))) & 1u)) x[16 * q + b] = -INFINITY;
+                    }
+                }
             }
+            // scores in base 2: x * sc (fp8: times each row's kv scale)
+            float sc = p.sc_log2;
+            if constexpr (kFp8) {
+#pragma unroll
+                for (int i = 0; i < 64; ++i) x[i] *= p.sc_log2 * cs[i];
+                sc = 1.0f;
+            }
+            float mx[8];
+#pragma unroll
+            for (int i = 0; i < 8; ++i)
+                mx[i] = fmaxf(fmaxf(fmaxf(x[8 * i], x[8 * i + 1]), fmaxf(x[8 * i + 2], x[8 * i + 3])),
+                              fmaxf(fmaxf(x[8 * i + 4], x[8 * i + 5]), fmaxf(x[8 * i + 6], x[8 * i + 7])));
+            const float m_tile = sc * fmaxf(fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])),
+                                            fmaxf(fmaxf(mx[4], mx[5]), fmaxf(mx[6], mx[7])));
             const float m_new = fmaxf(m_run, m_tile);
             const bool need = m_new > m_run + 8.0f;           // rescale only past 2^8 growth
             const float alpha = need ? fast_exp2(m_run - m_new) : 1.0f;
             if (need) m_run = m_new;
             const bool warp_rescale = __any_sync(0xffffffffu, need) && j > 0;
-            float lsum = 0.f;
+            const float msub = m_run == -INFINITY ? 0.f : m_run;   // exp2(-inf) = +0
+            float ls[4] = {0.f, 0.f, 0.f, 0.f};
             uint32_t pk[32];
 #pragma unroll
             for (int i = 0; i < 64; i += 2) {
-                const float e0 = (x[i] == -INFINITY) ? 0.f : fast_exp2(x[i] - m_run);
-                const float e1 = (x[i + 1] == -INFINITY) ? 0.f : fast_exp2(x[i + 1] - m_run);
-                lsum += e0 + e1;
+                const float e0 = fast_exp2(fmaf(x[i], sc, -msub));
+                const float e1 = fast_exp2(fmaf(x[i + 1], sc, -msub));
+                ls[(i >> 1) & 3] += e0 + e1;
                 pk[i / 2] = kFp8 ? pack_f16(e0 * cs[i], e1 * cs[i + 1]) : pack_f16(e0, e1);
             }
-            l_run = l_run * alpha + lsum;
-            // ---- O may be rescaled once PV(j-1) is done; P[j&1] is free once PV(j-2) is
-            if (warp_rescale && !mbar_wait(&pvdone[(j - 1) & 1], ((j - 1) >> 1) & 1, p.check)) {
-                alive = false;
-                break;
-            }
-            if (j >= 2 && !mbar_wait(&pvdone[j & 1], ((j - 2) >> 1) & 1, p.check)) { alive = false; break; }
+            l_run = l_run * alpha + ((ls[0] + ls[1]) + (ls[2] + ls[3]));
+            // ---- P (and O) are free once the previous PV has finished
+            if (j >= 1 && !mbar_wait_warp(pvdone, (j - 1) & 1, p.check)) { alive = false; break; }
             tc_fence_after();
             if (warp_rescale) {
 #pragma unroll 1
@@ -435,25 +451,20 @@ mla_tc_kernel(const Params p) {
                     for (int i = 0; i < 32; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * alpha);
                     tmem_st32(lane_base + kColO + cc * 32, o);
                 }
-                tmem_st_wait();
             }
-            const uint32_t prow = sb + kOffP + (j & 1) * kPBytes;
-#pragma unroll
-            for (int c8 = 0; c8 < 8; ++c8)
-                sts16(prow + sw128(h, c8), make_uint4(pk[4 * c8], pk[4 * c8 + 1], pk[4 * c8 + 2], pk[4 * c8 + 3]));
-            fence_proxy_async_smem();
+            tmem_st32(lane_base + kColP, pk);
+            tmem_st_wait();
             tc_fence_before();
-            mbar_arrive(&pfull[j & 1]);
+            mbar_arrive(pfull);
         }
-        // ---- epilogue: O_r / l and lse
-        const bool have = alive && n_tiles > 0 &&
-                          mbar_wait(&pvdone[(n_tiles - 1) & 1], ((n_tiles - 1) >> 1) & 1, p.check);
+        // ---- epilogue: O_v / l and lse
+        const bool have = alive && n_tiles > 0 && mbar_wait_warp(pvdone, (n_tiles - 1) & 1, p.check);
         tc_fence_after();
         const float inv = (have && l_run > 0.f) ? 1.0f / l_run : 0.f;
         const float lse_v = (have && l_run > 0.f) ? (m_run + log2f(l_run)) * 0.69314718055994531f
                                                   : -INFINITY;
         if (p.nsplit == 1) {
-            uint4* orow = reinterpret_cast<uint4*>(p.out + ((long long)t * kHeads + h) * 512 + rank * 256);
+            uint4* orow = reinterpret_cast<uint4*>(p.out + ((long long)t * kHeads + h) * 512 + vh * 256);
 #pragma unroll 1
             for (int cc = 0; cc < 8; ++cc) {
                 uint32_t o[32];
@@ -471,10 +482,10 @@ mla_tc_kernel(const Params p) {
                     orow[cc * 4 + q4] = w;
                 }
             }
-            if (rank == 0 && p.lse) p.lse[(long long)t * kHeads + h] = lse_v;
+            if (vh == 0 && p.lse) p.lse[(long long)t * kHeads + h] = lse_v;
         } else {
             const long long pb = ((long long)t * p.nsplit + split) * kHeads + h;
-            float4* orow = reinterpret_cast<float4*>(p.o_part + pb * 512 + rank * 256);
+            float4* orow = reinterpret_cast<float4*>(p.o_part + pb * 512 + vh * 256);
 #pragma unroll 1
             for (int cc = 0; cc < 8; ++cc) {
                 uint32_t o[32];
@@ -490,13 +501,12 @@ mla_tc_kernel(const Params p) {
                                                            __uint_as_float(o[4 * q4 + 3]) * inv)
                                              : make_float4(0.f, 0.f, 0.f, 0.f);
             }
-            if (rank == 0) p.lse_part[pb] = lse_v;
+            if (vh == 0) p.lse_part[pb] = lse_v;
         }
     }
 
     tc_fence_before();
     __syncthreads();
-    cluster_sync();   // no remote shared-memory traffic after this point
     tc_fence_after();
     if (warp == kMmaWarp) tmem_dealloc(tmem, kTmemCols);
 }
