@@ -186,6 +186,8 @@ dsa_status_t mla_check(const void* q, dsa_dtype_t q_dtype, int heads, int d_qk, 
         if (heads != 128 || d_qk != 576 || d_v != 512)
             return fail(DSA_ERR_UNSUPPORTED, "bf16 sparse MLA supports heads = 128, d_qk = 576, d_v = 512");
         if (out_dtype != DSA_BF16) return fail(DSA_ERR_UNSUPPORTED, "bf16 sparse MLA writes bf16 output");
+        if (plan->kv.num_pages >= 0x7FFFFFFFLL)
+            return fail(DSA_ERR_UNSUPPORTED, "latent KV caches are limited to 2^31 - 1 rows");
         plan->kind = MlaKind::kTensorCore;
         return DSA_OK;
     }

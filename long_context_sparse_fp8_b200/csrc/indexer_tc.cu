@@ -19,10 +19,6 @@
 // Grid: x = groups of G consecutive query rows (G = 1 for decode-like batches,
 // 4 otherwise; a group that spans sequences is processed as per-sequence runs),
 // y = chunks of the key tiles, so that short batches still cover all SMs.
-#include <cudaTypedefs.h>
-
-#include <mutex>
-
 #include "kernels.h"
 #include "sm100.cuh"
 
@@ -305,31 +301,10 @@ indexer_fp8_tc_kernel(const __grid_constant__ CUtensorMap tm_k,
     if (warp == 1) tmem_dealloc(tmem_base, tmem_cols);
 }
 
-PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
-    static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
-    static std::once_flag once;
-    std::call_once(once, [] {
-        void* ptr = nullptr;
-        cudaDriverEntryPointQueryResult q;
-        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) ==
-                cudaSuccess && q == cudaDriverEntryPointSuccess)
-            fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(ptr);
-    });
-    return fn;
-}
-
 // 2-D byte matrix [rows][128] with a 128 x box_rows box, 128-byte swizzle.
 cudaError_t make_map(CUtensorMap* m, const void* base, unsigned long long rows, uint32_t box_rows) {
-    auto fn = encode_fn();
-    if (!fn) return cudaErrorNotSupported;
-    cuuint64_t dims[2] = {128, rows};
-    cuuint64_t strides[1] = {128};
-    cuuint32_t box[2] = {128, box_rows};
-    cuuint32_t estr[2] = {1, 1};
-    CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(base), dims, strides,
-                    box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
-                    CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
-    return r == CUDA_SUCCESS ? cudaSuccess : cudaErrorInvalidValue;
+    return make_tensor_map_2d(m, base, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, 128, rows, 128, 128,
+                              box_rows, CU_TENSOR_MAP_SWIZZLE_128B);
 }
 
 }  // namespace

@@ -2,6 +2,7 @@
 // in include/dsa.h validates arguments and then calls these.
 #pragma once
 
+#include <cuda.h>
 #include <cuda_runtime.h>
 
 #include "common.cuh"
@@ -10,6 +11,12 @@ namespace dsa {
 
 constexpr int kIndexerPage = 64;
 constexpr int kNumSMs = 148;
+
+// 2-D tensor map [rows][inner] (row stride in bytes) with a box_inner x box_rows box.
+cudaError_t make_tensor_map_2d(CUtensorMap* m, const void* base, CUtensorMapDataType dtype,
+                               int elem_bytes, unsigned long long inner, unsigned long long rows,
+                               unsigned long long row_stride_bytes, unsigned box_inner,
+                               unsigned box_rows, CUtensorMapSwizzle swizzle);
 
 // Lightning Indexer on CUDA cores (fp32 q/k; any heads <= 64, dim <= 128, dim % 4 == 0).
 cudaError_t launch_indexer_generic(const void* q, const float* q_scale, const float* w, int heads,
