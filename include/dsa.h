@@ -173,6 +173,46 @@ DSA_API dsa_status_t dsa_sparse_mla_decode(const void* q, dsa_dtype_t q_dtype, i
                                            size_t workspace_bytes, dsa_stream_t stream);
 
 /*
+ * dsa_sparse_mla_decode_noalloc -- dsa_sparse_mla_decode for callers that cannot
+ * hand over a workspace: the split partials go to a fixed array that the library
+ * holds in device memory (a file-scope __device__ array of
+ * DSA_NOALLOC_SCRATCH_BYTES per device) instead.  This call is an addition of
+ * this library; the DeepSeek-V3.2 pages describe no such variant.
+ *
+ * Who needs it: a caller with no device allocator of its own (a plain C host
+ * program, a plug-in that must not touch the host framework's memory pool), or
+ * one that has committed every free byte of HBM to its KV caches at start-up
+ * and so has no room left to carve a workspace from.  Nothing in the call
+ * allocates or frees device memory; the array is set aside by the CUDA runtime
+ * when the library's module holding it is loaded on the device.
+ *
+ * Limits and rules:
+ *   - dsa_sparse_mla_decode_workspace_size(total_q, heads, d_v, k) must not
+ *     exceed DSA_NOALLOC_SCRATCH_BYTES (20 MiB); a larger need returns
+ *     DSA_ERR_WORKSPACE_TOO_SMALL with a message and queues nothing.  The split
+ *     rule of this version keeps rows x splits <= 74, so its largest need is
+ *     74 x 128 heads x 512 x 4 B plus the lse (19.4 MB) and every call the
+ *     kernels accept fits (32 decode rows at k = 2048 need 16.03 MiB).
+ *   - The first call on each device looks the array's address up (with that
+ *     device current) and caches it; make that first call before beginning any
+ *     stream capture.
+ *   - There is one array per device: two calls on one device whose executions
+ *     may overlap (different streams not ordered by events, or different host
+ *     threads) race on it and give wrong results.  Calls on one stream are safe.
+ *   - The array keeps whatever the last call left in it.  Every call writes each
+ *     partial it reads before reading it, so nothing needs to start at zero.
+ * Other arguments, the kernels used and the results are those of
+ * dsa_sparse_mla_decode.
+ */
+#define DSA_NOALLOC_SCRATCH_BYTES ((size_t)20 << 20)
+DSA_API dsa_status_t dsa_sparse_mla_decode_noalloc(const void* q, dsa_dtype_t q_dtype,
+                                                   int32_t heads, int32_t d_qk, int32_t d_v,
+                                                   float softmax_scale, const dsa_paged_cache_t* kv,
+                                                   const dsa_batch_t* batch, const int32_t* idx,
+                                                   int32_t k, void* out, dsa_dtype_t out_dtype,
+                                                   float* lse, dsa_stream_t stream);
+
+/*
  * dsa_decode -- the whole decode step in one call: indexer logits -> top-k ->
  * sparse MLA (split + merge), queued back to back on `stream`.  The logits and
  * the index lists live in the workspace; idx_out (nullable, [T][k]) receives a

@@ -343,6 +343,39 @@ DSA_API dsa_status_t dsa_sparse_mla_decode(const void* q, dsa_dtype_t q_dtype, i
     return e == cudaSuccess ? ok() : cuda_fail(e, "sparse MLA decode launch");
 }
 
+DSA_API dsa_status_t dsa_sparse_mla_decode_noalloc(const void* q, dsa_dtype_t q_dtype,
+                                                   int32_t heads, int32_t d_qk, int32_t d_v,
+                                                   float softmax_scale, const dsa_paged_cache_t* kv,
+                                                   const dsa_batch_t* batch, const int32_t* idx,
+                                                   int32_t k, void* out, dsa_dtype_t out_dtype,
+                                                   float* lse, dsa_stream_t stream) {
+    static_assert(kStaticScratchBytes == DSA_NOALLOC_SCRATCH_BYTES, "scratch size mismatch");
+    BatchView bv;
+    MlaPlan plan;
+    dsa_status_t s = check_batch(batch, &bv);
+    if (s != DSA_OK || bv.total_q == 0) return s == DSA_OK ? ok() : s;
+    s = mla_check(q, q_dtype, heads, d_qk, d_v, softmax_scale, kv, bv, idx, k, out, out_dtype,
+                  lse, &plan);
+    if (s != DSA_OK) return s;
+    const size_t need = mla_decode_ws(bv.total_q, heads, d_v, k);
+    if (need > kStaticScratchBytes)
+        return fail(DSA_ERR_WORKSPACE_TOO_SMALL,
+                    "dsa_sparse_mla_decode_noalloc: this batch needs %zu bytes of split scratch "
+                    "but the built-in array holds %zu; use dsa_sparse_mla_decode with a workspace",
+                    need, kStaticScratchBytes);
+    int* check = nullptr;
+    void* scratch = nullptr;
+    cudaError_t e = check_word(&check);
+    if (e != cudaSuccess) return cuda_fail(e, "check word address");
+    if (need) {
+        e = static_scratch(&scratch);
+        if (e != cudaSuccess) return cuda_fail(e, "static scratch address");
+    }
+    e = mla_decode_launch(plan, q, heads, d_qk, d_v, softmax_scale, bv, idx, k, out, out_dtype, lse,
+                          scratch, check, static_cast<cudaStream_t>(stream));
+    return e == cudaSuccess ? ok() : cuda_fail(e, "sparse MLA decode (static scratch) launch");
+}
+
 DSA_API size_t dsa_decode_workspace_size(const dsa_batch_t* batch, int32_t k, int32_t heads,
                                          int32_t d_v) {
     if (!batch || batch->total_q < 0 || batch->max_seq_len < 1 || k < 1 || heads < 1 || d_v < 1)

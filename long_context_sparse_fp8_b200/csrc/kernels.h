@@ -44,6 +44,13 @@ cudaError_t launch_mla_tc(const void* q, float scale, const CacheView& kv, const
                           const int* idx, int k, int nsplit, void* out, float* lse, float* o_part,
                           float* lse_part, int* check, cudaStream_t st);
 
+// Size of the fixed device array behind dsa_sparse_mla_decode_noalloc
+// (equals DSA_NOALLOC_SCRATCH_BYTES in include/dsa.h).
+constexpr size_t kStaticScratchBytes = size_t(20) << 20;
+
+// Address of that array on the current device (looked up once per device).
+cudaError_t static_scratch(void** ptr);
+
 // Log-sum-exp merge of split partials into out (out_dtype) and lse.
 cudaError_t launch_mla_combine(const float* o_part, const float* lse_part, int total_q, int nsplit,
                                int heads, int d_v, void* out, int out_dtype, float* lse,

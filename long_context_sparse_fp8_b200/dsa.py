@@ -30,6 +30,7 @@ DSA_FP8_E4M3 = 2
 EXPORTED = (
     "dsa_indexer_logits", "dsa_topk", "dsa_sparse_mla_prefill",
     "dsa_sparse_mla_decode_workspace_size", "dsa_sparse_mla_decode",
+    "dsa_sparse_mla_decode_noalloc",
     "dsa_decode_workspace_size", "dsa_decode", "dsa_device_check", "dsa_last_error_message",
     "dsa_status_string", "dsa_version",
 )
@@ -79,6 +80,8 @@ def load_library(path: str = _LIB_PATH) -> ctypes.CDLL:
         "dsa_sparse_mla_decode_workspace_size": ([i32, i32, i32, i32], sz),
         "dsa_sparse_mla_decode": ([P, ctypes.c_int, i32, i32, i32, f32, CP, BP, P, i32, P,
                                    ctypes.c_int, P, P, sz, P], ctypes.c_int),
+        "dsa_sparse_mla_decode_noalloc": ([P, ctypes.c_int, i32, i32, i32, f32, CP, BP, P, i32,
+                                           P, ctypes.c_int, P, P], ctypes.c_int),
         "dsa_decode_workspace_size": ([BP, i32, i32, i32], sz),
         "dsa_decode": ([P, ctypes.c_int, P, P, i32, i32, CP, i32, P, ctypes.c_int, i32, i32, i32,
                         f32, CP, BP, P, P, ctypes.c_int, P, P, sz, P], ctypes.c_int),
@@ -193,6 +196,22 @@ def dsa_sparse_mla_decode(q, kv: PagedCache, batch: Batch, idx, d_v: int, softma
         _ptr(q), dtype_code(q), heads, d_qk, int(d_v), float(softmax_scale), ctypes.byref(kc),
         ctypes.byref(bc), _ptr(idx), int(idx.shape[-1]), _ptr(out), dtype_code(out), _ptr(lse),
         _ptr(workspace), ws_bytes, _stream(stream)))
+    return out
+
+
+DSA_NOALLOC_SCRATCH_BYTES = 20 << 20
+
+
+def dsa_sparse_mla_decode_noalloc(q, kv: PagedCache, batch: Batch, idx, d_v: int,
+                                  softmax_scale: float, out, lse=None, stream=None):
+    """dsa_sparse_mla_decode with the split partials in the library's fixed device
+    array (no workspace argument; calls whose executions overlap on one device race)."""
+    heads, d_qk = int(q.shape[-2]), int(q.shape[-1])
+    kc, bc = kv.c(), batch.c()
+    _check(load_library().dsa_sparse_mla_decode_noalloc(
+        _ptr(q), dtype_code(q), heads, d_qk, int(d_v), float(softmax_scale), ctypes.byref(kc),
+        ctypes.byref(bc), _ptr(idx), int(idx.shape[-1]), _ptr(out), dtype_code(out), _ptr(lse),
+        _stream(stream)))
     return out
 
 
