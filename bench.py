@@ -24,6 +24,7 @@ import os
 import statistics
 import subprocess
 import sys
+import threading
 import time
 
 import torch
@@ -47,8 +48,8 @@ WORKLOADS = {
 def parse():
     p = argparse.ArgumentParser()
     p.add_argument("--gpus", type=int, default=1)
-    p.add_argument("--steps", type=int, default=20)
-    p.add_argument("--warmup", type=int, default=5)
+    p.add_argument("--steps", type=int, default=200)
+    p.add_argument("--warmup", type=int, default=10)
     p.add_argument("--impl", choices=["dsa", "reference"], default="dsa")
     p.add_argument("--workload", choices=sorted(WORKLOADS), default="decode_b32_ctx8192")
     p.add_argument("--no-cpu-baseline", action="store_true")
@@ -85,7 +86,10 @@ def max_over_ranks(x: float, world: int) -> float:
 
 
 class ClockSampler:
-    """nvidia-smi clocks / throttle reasons sampled every 200 ms during the timed loop."""
+    """SM clock and clock-event reasons of this process's GPU, read through NVML every
+    millisecond or so by a background thread while the timed loop runs (the loop lasts
+    only milliseconds, so nvidia-smi's 200 ms period would miss it).  Falls back to
+    nvidia-smi when NVML is unavailable."""
     Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
          "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
          "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
@@ -93,8 +97,39 @@ class ClockSampler:
     def __init__(self, gpu_index: int):
         self.gpu = gpu_index
         self.proc = None
+        self.thread = None
+        self.samples = []        # (sm_mhz, reason bits)
+        self.lines = []
+        self.smax = None
+
+    def _nvml_handle(self):
+        import pynvml
+        pynvml.nvmlInit()
+        pr = torch.cuda.get_device_properties(self.gpu)
+        bus = f"{pr.pci_domain_id:08X}:{pr.pci_bus_id:02X}:{pr.pci_device_id:02X}.0"
+        return pynvml, pynvml.nvmlDeviceGetHandleByPciBusId(bus)
 
     def __enter__(self):
+        try:
+            nv, h = self._nvml_handle()
+            self.smax = float(nv.nvmlDeviceGetMaxClockInfo(h, nv.NVML_CLOCK_SM))
+            self.stop = threading.Event()
+
+            def poll():
+                while not self.stop.is_set():
+                    try:
+                        self.samples.append((nv.nvmlDeviceGetClockInfo(h, nv.NVML_CLOCK_SM),
+                                             nv.nvmlDeviceGetCurrentClocksEventReasons(h)))
+                    except Exception:  # noqa: BLE001 -- sampling must never fail the run
+                        pass
+                    time.sleep(0.001)
+
+            self.thread = threading.Thread(target=poll, daemon=True)
+            self.thread.start()
+            time.sleep(0.005)
+            return self
+        except Exception:  # noqa: BLE001
+            self.thread = None
         try:
             self.proc = subprocess.Popen(
                 ["nvidia-smi", f"--id={self.gpu}", f"--query-gpu={self.Q}",
@@ -105,7 +140,9 @@ class ClockSampler:
         return self
 
     def __exit__(self, *exc):
-        self.lines = []
+        if self.thread is not None:
+            self.stop.set()
+            self.thread.join(timeout=5)
         if self.proc is not None:
             time.sleep(0.25)
             self.proc.terminate()
@@ -116,10 +153,18 @@ class ClockSampler:
                 out, _ = self.proc.communicate()
             self.lines = [ln for ln in out.splitlines() if ln.strip()]
 
+    BITS = {"hw_slowdown": 0x8, "hw_thermal_slowdown": 0x40, "sw_thermal_slowdown": 0x20,
+            "sw_power_cap": 0x4}
+
     def summary(self):
-        sm, smax, reasons = [], None, set()
+        sm, smax, reasons = [], self.smax, set()
+        for mhz, bits in self.samples:
+            sm.append(float(mhz))
+            for n, b in self.BITS.items():
+                if bits & b:
+                    reasons.add(n)
         names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        for ln in getattr(self, "lines", []):
+        for ln in self.lines:
             f = [x.strip() for x in ln.split(",")]
             if len(f) < 9:
                 continue
@@ -132,9 +177,9 @@ class ClockSampler:
                 if v.lower().startswith("active"):
                     reasons.add(n)
         if not sm:
-            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unsampled"]}
+            return {"sm_mhz": None, "sm_max_mhz": smax, "reasons": ["unsampled"]}
         return {"sm_mhz": statistics.median(sm), "sm_max_mhz": smax, "reasons": sorted(reasons),
-                "samples": len(sm)}
+                "samples": len(sm), "source": "nvml" if self.samples else "nvidia-smi"}
 
 
 def measured_peaks():
@@ -146,8 +191,9 @@ def measured_peaks():
         return 6650.0, 1590.0, "fallback"
 
 
-def ncu_traffic(kernel_file: str):
-    """DRAM bytes per launch from the committed ncu summary, if the kernel is unchanged."""
+def ncu_traffic(workload: str, kernel_file: str):
+    """DRAM bytes per launch from the committed ncu summary of this workload, if the
+    kernel source is unchanged since the capture."""
     path = os.path.join(ROOT, "profiles", "ncu_traffic.json")
     try:
         with open(path) as f:
@@ -159,7 +205,7 @@ def ncu_traffic(kernel_file: str):
         sha = hashlib.sha256(open(src, "rb").read()).hexdigest()[:16]
     except OSError:
         return None
-    entry = rec.get(kernel_file)
+    entry = rec.get(workload, {}).get(kernel_file)
     if not entry or entry.get("source_sha") != sha:
         return None
     return entry.get("dram_bytes_per_launch")
@@ -296,9 +342,8 @@ def run_dsa(args, rank, world):
         peak = bf16_tf * (2.0 if dom == "indexer" else 1.0)
         roof = {"bound": "tensor", "achieved": round(fl, 1), "peak": peak, "unit": "TFLOP/s"}
     roof["frac"] = round(roof["achieved"] / roof["peak"], 4)
-    kernel_file = {"indexer": "indexer_generic.cu", "topk": "topk.cu",
-                   "mla": "mla_generic.cu"}[dom]
-    roof["traffic"] = ncu_traffic(kernel_file)
+    kernel_file = {"indexer": "indexer_tc.cu", "topk": "topk.cu", "mla": "mla_tc.cu"}[dom]
+    roof["traffic"] = ncu_traffic(args.workload, kernel_file)
     roof["kernel"] = dom
     roof["peak_source"] = f"{peak_kind} ({'burst' if roof['unit'] == 'GB/s' else 'burst bf16'})"
     roof["stage_ms"] = {n: round(v, 4) for n, v in mean_stage.items()}
