@@ -4,12 +4,26 @@
 // "DeepSeek Sparse Attention").  A row with pos+1 <= k keeps every position
 // (dense fallback, same guide, section 5.1).
 //
-// Method: exact radix select on order-preserving 32-bit keys.  One 1024-thread CTA
-// owns one row.  Three histogram passes (11 + 11 + 10 bits, shared-memory
-// atomics) pin down the exact k-th largest key T and how many keys equal to T
-// are still needed; a final two-pass emission writes every key > T and the
-// lowest-position keys == T in ascending position order (deterministic output).  Rows of up to kSmemKeys candidates are staged once in shared
-// memory; longer rows are re-read from global memory (L2) on each pass.
+// Method: exact radix select on order-preserving 32-bit keys, one 1024-thread CTA
+// per row, output in ascending position order (deterministic; equal keys at the
+// threshold go to the lowest positions).
+//
+//   1. One vectorised read of the row stages the keys in shared memory (up to the
+//      staging capacity; the rest is re-read from L2) and builds a histogram of the
+//      top 11 key bits.  Logits crowd into a few exponent bins, so each lane adds to
+//      one of four interleaved histogram copies to cut same-address conflicts.  The
+//      histogram fixes the bin b1 of the k-th key: every key in a higher bin is in.
+//   2. One sweep over 32-key groups writes a selection bitmap straight from warp
+//      ballots (bit set = bin above b1) and appends the keys of bin b1 with their
+//      positions to a candidate list C.
+//   3. Two radix passes (11 + 10 bits) over C fix the exact k-th key T and how many
+//      keys equal to T are needed; keys above T get their bit, and the equal keys
+//      go to a second bitmap from which the lowest positions are taken.
+//   4. A block scan over the bitmap's popcounts turns it into the ascending list.
+// If C would overflow (thousands of keys in one bin, e.g. equal scores), step 2 is
+// replaced by radix passes over the whole row and one marking sweep.  Rows longer
+// than the bitmap capacity use a second kernel that refines over the whole row and
+// emits in two ordered sweeps.
 #include "kernels.h"
 
 namespace dsa {
@@ -17,7 +31,13 @@ namespace {
 
 constexpr int kThreads = 1024;
 constexpr int kWarps = kThreads / 32;
-constexpr int kSmemKeys = 48 * 1024;  // 192 KB of staged keys
+constexpr int kTopBits = 11;
+constexpr uint32_t kLowMask = (1u << (32 - kTopBits)) - 1u;   // 21 low key bits
+constexpr int kCopies = 4;                 // interleaved copies of the first histogram
+constexpr int kCandCap = 4096;             // candidates: low 21 key bits + position
+constexpr int kMaxWords = 8192;            // bitmap words: rows up to 262144 keys
+constexpr int kSmemLimit = 232448;
+constexpr int kStaticReserve = 1024;
 
 // Monotone map float -> uint32 (larger float, larger key); -0.0 maps like +0.0.
 __device__ __forceinline__ uint32_t order_key(float f) {
@@ -26,8 +46,13 @@ __device__ __forceinline__ uint32_t order_key(float f) {
     return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
 }
 
+struct Shared {
+    int warp_sums[kWarps + 1];
+    int bin, above, count, n_c;
+};
+
 // Block-wide exclusive prefix sum of one int per thread; *total gets the sum.
-__device__ __forceinline__ int block_excl_scan(int v, int* warp_sums, int* total) {
+__device__ __forceinline__ int block_excl_scan(int v, Shared& sh, int* total) {
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     int x = v;
 #pragma unroll
@@ -35,43 +60,161 @@ __device__ __forceinline__ int block_excl_scan(int v, int* warp_sums, int* total
         int y = __shfl_up_sync(0xffffffffu, x, o);
         if (lane >= o) x += y;
     }
-    if (lane == 31) warp_sums[warp] = x;
+    if (lane == 31) sh.warp_sums[warp] = x;
     __syncthreads();
     if (warp == 0) {
-        int w = warp_sums[lane];
+        int w = sh.warp_sums[lane];
         int s = w;
 #pragma unroll
         for (int o = 1; o < 32; o <<= 1) {
             int y = __shfl_up_sync(0xffffffffu, s, o);
             if (lane >= o) s += y;
         }
-        warp_sums[lane] = s - w;        // exclusive per warp
-        if (lane == 31) warp_sums[32] = s;
+        sh.warp_sums[lane] = s - w;        // exclusive per warp
+        if (lane == 31) sh.warp_sums[32] = s;
     }
     __syncthreads();
-    const int r = warp_sums[warp] + x - v;
-    *total = warp_sums[32];
+    const int r = sh.warp_sums[warp] + x - v;
+    *total = sh.warp_sums[32];
     __syncthreads();  // warp_sums may be reused right after
     return r;
 }
 
+// The bin (of nb = 1024 or 2048, counted from the top) holding the remaining-th
+// largest key, summing `copies` histograms spaced 2048 apart; *above = keys in
+// higher bins, *count = keys in the bin.  Ends synchronised.
+__device__ __forceinline__ int find_bin(Shared& sh, const int* hist, int copies, int nb,
+                                        int remaining, int* above, int* count) {
+    const int tid = threadIdx.x;
+    const int per = nb / kThreads;
+    int local[2] = {0, 0};
+#pragma unroll
+    for (int j = 0; j < 2; ++j) {
+        if (j < per) {
+            const int bin = nb - 1 - (tid * per + j);
+            for (int c = 0; c < copies; ++c) local[j] += hist[c * 2048 + bin];
+        }
+    }
+    int total;
+    int run = block_excl_scan(local[0] + local[1], sh, &total);
+#pragma unroll
+    for (int j = 0; j < 2; ++j) {
+        if (j < per) {
+            const int ab = run;
+            run += local[j];
+            if (run >= remaining && ab < remaining) {
+                sh.bin = nb - 1 - (tid * per + j);
+                sh.above = ab;
+                sh.count = local[j];
+            }
+        }
+    }
+    __syncthreads();
+    *above = sh.above;
+    *count = sh.count;
+    const int b = sh.bin;
+    __syncthreads();
+    return b;
+}
+
+// Keys of the row: staged prefix in shared memory, the rest re-read from global.
 struct Row {
-    const float* g;       // global row
-    const uint32_t* s;    // staged keys or nullptr
+    const float* g;
+    const uint32_t* s;
+    int cap;
     __device__ __forceinline__ uint32_t operator()(int i) const {
-        return s ? s[i] : order_key(__ldg(g + i));
+        return i < cap ? s[i] : order_key(__ldg(g + i));
     }
 };
 
-__global__ void __launch_bounds__(kThreads)
-topk_kernel(const float* __restrict__ logits, long long ld, BatchView bv, int k,
-            int* __restrict__ idx, int* check, int smem_keys) {
-    extern __shared__ uint32_t skeys[];
-    __shared__ int hist[2048];
-    __shared__ int warp_sums[kWarps + 1];
-    __shared__ int s_bin, s_above;
+// One radix refinement pass over n keys: histogram (copy 0) of bits
+// [shift, shift+nbits) of the keys matching prefix/pmask, then the bin of the
+// remaining-th largest; *count = keys in that bin.
+template <class KeyF>
+__device__ __forceinline__ void refine(Shared& sh, int* hist, int n, KeyF key_of, int shift,
+                                       int nbits, uint32_t& prefix, uint32_t& pmask,
+                                       int& remaining, int* count) {
+    const int nb = 1 << nbits, tid = threadIdx.x;
+    for (int i = tid; i < nb; i += kThreads) hist[i] = 0;
+    __syncthreads();
+    for (int i = tid; i < n; i += kThreads) {
+        const uint32_t key = key_of(i);
+        if ((key & pmask) == prefix) atomicAdd(&hist[(key >> shift) & (nb - 1)], 1);
+    }
+    __syncthreads();
+    int above;
+    const int bin = find_bin(sh, hist, 1, nb, remaining, &above, count);
+    remaining -= above;
+    prefix |= (uint32_t)bin << shift;
+    pmask |= (uint32_t)(nb - 1) << shift;
+}
 
-    const int t = blockIdx.x, tid = threadIdx.x;
+// Stage the row's keys (first `cap`) and build the interleaved top-bit histogram.
+__device__ __forceinline__ void stage_and_histogram(const float* grow, int n, uint32_t* skeys,
+                                                    int cap, int* hist) {
+    const int tid = threadIdx.x;
+    int* my_hist = hist + (tid & (kCopies - 1)) * 2048;
+    for (int base = 0; base < n; base += 8 * kThreads) {
+        float v[8];
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+            const int i0 = base + h * 4 * kThreads + 4 * tid;
+            if (i0 + 3 < n) {
+                const float4 f = __ldg(reinterpret_cast<const float4*>(grow + i0));
+                v[4 * h] = f.x; v[4 * h + 1] = f.y; v[4 * h + 2] = f.z; v[4 * h + 3] = f.w;
+            } else {
+#pragma unroll
+                for (int j = 0; j < 4; ++j) v[4 * h + j] = i0 + j < n ? __ldg(grow + i0 + j) : 0.f;
+            }
+        }
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+                const int i = base + h * 4 * kThreads + 4 * tid + j;
+                if (i < n) {
+                    const uint32_t key = order_key(v[4 * h + j]);
+                    if (i < cap) skeys[i] = key;
+                    atomicAdd(&my_hist[key >> (32 - kTopBits)], 1);
+                }
+            }
+        }
+    }
+}
+
+// Bitmap of the selected positions (ascending) -> out[0, count).
+__device__ __forceinline__ void bitmap_to_list(Shared& sh, const uint32_t* bits, int words,
+                                               int* out) {
+    const int tid = threadIdx.x;
+    const int wpt = (words + kThreads - 1) / kThreads;
+    const int w0 = min(words, tid * wpt), w1 = min(words, w0 + wpt);
+    int c = 0;
+    for (int w = w0; w < w1; ++w) c += __popc(bits[w]);
+    int total;
+    int at = block_excl_scan(c, sh, &total);
+    for (int w = w0; w < w1; ++w) {
+        uint32_t b = bits[w];
+        while (b) {
+            const int bit = __ffs(b) - 1;
+            out[at++] = 32 * w + bit;
+            b &= b - 1u;
+        }
+    }
+}
+
+__global__ void __launch_bounds__(kThreads, 1)
+topk_kernel(const float* __restrict__ logits, long long ld, BatchView bv, int k,
+            int* __restrict__ idx, int* check, int words_cap, int stage_cap) {
+    extern __shared__ __align__(16) uint8_t dyn[];
+    int* hist = reinterpret_cast<int*>(dyn);                                   // [4][2048]
+    uint32_t* ckey = reinterpret_cast<uint32_t*>(dyn + kCopies * 2048 * 4);      // [kCandCap]
+    int* cpos = reinterpret_cast<int*>(ckey + kCandCap);                         // [kCandCap]
+    uint32_t* bitmap = reinterpret_cast<uint32_t*>(cpos + kCandCap);             // [words_cap]
+    uint32_t* eqmap = bitmap + words_cap;                                        // [words_cap]
+    uint32_t* skeys = eqmap + words_cap;                                         // [stage_cap]
+    __shared__ Shared sh;
+
+    const int t = blockIdx.x, tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     int* out = idx + (long long)t * k;
     const RowInfo ri = row_info(bv, t, check);
     if (!ri.ok) {
@@ -84,63 +227,164 @@ topk_kernel(const float* __restrict__ logits, long long ld, BatchView bv, int k,
         return;
     }
     const float* grow = logits + (long long)t * ld;
-    Row row{grow, nullptr};
-    if (n <= smem_keys) {
-        for (int i = tid; i < n; i += kThreads) skeys[i] = order_key(__ldg(grow + i));
-        row.s = skeys;
-        __syncthreads();
-    }
+    const Row row{grow, skeys, stage_cap};
+    const int words = (n + 31) >> 5;
 
-    // ---- radix select: find the exact k-th largest key -------------------------
-    uint32_t prefix = 0u, pmask = 0u;
-    int remaining = k;   // how many of the keys matching `prefix` still have to be taken
-    const int shifts[3] = {21, 10, 0};
-    const int nbits[3] = {11, 11, 10};
-#pragma unroll 1
-    for (int p = 0; p < 3; ++p) {
-        const int nb = 1 << nbits[p], shift = shifts[p];
-        for (int i = tid; i < nb; i += kThreads) hist[i] = 0;
-        __syncthreads();
-        for (int i = tid; i < n; i += kThreads) {
-            const uint32_t key = row(i);
-            if ((key & pmask) == prefix) atomicAdd(&hist[(key >> shift) & (nb - 1)], 1);
-        }
-        __syncthreads();
-        // Suffix counts from the top bin down: thread tid owns reversed bins
-        // [tid*per, tid*per + per).
-        const int per = nb / kThreads;
-        int local[2] = {0, 0};
-        int tsum = 0;
-        for (int j = 0; j < per; ++j) {
-            local[j] = hist[nb - 1 - (tid * per + j)];
-            tsum += local[j];
-        }
-        int total;
-        int run = block_excl_scan(tsum, warp_sums, &total);
-        for (int j = 0; j < per; ++j) {
-            const int bin = nb - 1 - (tid * per + j);
-            const int above = run;
-            run += local[j];
-            if (run >= remaining && above < remaining) {
-                s_bin = bin;
-                s_above = above;
+    // ---- 1. stage + top-bit histogram ------------------------------------------
+    for (int i = tid; i < kCopies * 2048; i += kThreads) hist[i] = 0;
+    if (tid == 0) sh.n_c = 0;
+    __syncthreads();
+    stage_and_histogram(grow, n, skeys, stage_cap, hist);
+    __syncthreads();
+    int n_def, n_cand;
+    const uint32_t b1 = (uint32_t)find_bin(sh, hist, kCopies, 2048, k, &n_def, &n_cand);
+    int remaining = k - n_def;          // keys of bin b1 still to take (>= 1)
+    uint32_t T;                         // the k-th largest key
+    int n_eq;                           // keys equal to T
+
+    if (n_cand <= kCandCap) {
+        // ---- 2. bitmap of the higher bins; candidates of bin b1 -> C -------------
+        for (int g0 = warp; g0 < words; g0 += 4 * kWarps) {
+            uint32_t kk[4];
+#pragma unroll
+            for (int u = 0; u < 4; ++u) {
+                const int i = 32 * (g0 + u * kWarps) + lane;
+                kk[u] = i < n ? row(i) : 0u;
+            }
+#pragma unroll
+            for (int u = 0; u < 4; ++u) {
+                const int g = g0 + u * kWarps;
+                if (g >= words) break;
+                const int i = 32 * g + lane;
+                const uint32_t bin = kk[u] >> (32 - kTopBits);
+                const unsigned md = __ballot_sync(0xffffffffu, i < n && bin > b1);
+                const bool cand = i < n && bin == b1;
+                const unsigned mc = __ballot_sync(0xffffffffu, cand);
+                if (lane == 0) {
+                    bitmap[g] = md;
+                    eqmap[g] = 0u;
+                }
+                if (mc) {
+                    int base = 0;
+                    if (lane == 0) base = atomicAdd(&sh.n_c, __popc(mc));
+                    base = __shfl_sync(0xffffffffu, base, 0);
+                    if (cand) {
+                        const int c = base + __popc(mc & ((1u << lane) - 1u));
+                        ckey[c] = kk[u] & kLowMask;
+                        cpos[c] = i;
+                    }
+                }
             }
         }
         __syncthreads();
-        const int bin = s_bin;
-        remaining -= s_above;
-        prefix |= (uint32_t)bin << shift;
-        pmask |= (uint32_t)(nb - 1) << shift;
-        __syncthreads();
+        // ---- 3. exact threshold among the candidates; mark them ------------------
+        uint32_t prefix = 0u, pmask = 0u;
+        auto cand_key = [&](int i) { return ckey[i]; };
+        refine(sh, hist, n_cand, cand_key, 10, 11, prefix, pmask, remaining, &n_eq);
+        refine(sh, hist, n_cand, cand_key, 0, 10, prefix, pmask, remaining, &n_eq);
+        T = prefix;
+        for (int c = tid; c < n_cand; c += kThreads) {
+            const uint32_t key = ckey[c];
+            const int p = cpos[c];
+            if (key > T) atomicOr(&bitmap[p >> 5], 1u << (p & 31));
+            else if (key == T) atomicOr(&eqmap[p >> 5], 1u << (p & 31));
+        }
+    } else {
+        // ---- fallback: refine over the whole row, then one marking sweep ---------
+        uint32_t prefix = b1 << (32 - kTopBits);
+        uint32_t pmask = ~kLowMask;
+        refine(sh, hist, n, row, 10, 11, prefix, pmask, remaining, &n_eq);
+        refine(sh, hist, n, row, 0, 10, prefix, pmask, remaining, &n_eq);
+        T = prefix;
+        for (int g0 = warp; g0 < words; g0 += 4 * kWarps) {
+            uint32_t kk[4];
+#pragma unroll
+            for (int u = 0; u < 4; ++u) {
+                const int i = 32 * (g0 + u * kWarps) + lane;
+                kk[u] = i < n ? row(i) : 0u;
+            }
+#pragma unroll
+            for (int u = 0; u < 4; ++u) {
+                const int g = g0 + u * kWarps;
+                if (g >= words) break;
+                const int i = 32 * g + lane;
+                const unsigned mg = __ballot_sync(0xffffffffu, i < n && kk[u] > T);
+                const unsigned me = __ballot_sync(0xffffffffu, i < n && kk[u] == T);
+                if (lane == 0) {
+                    bitmap[g] = mg;
+                    eqmap[g] = me;
+                }
+            }
+        }
     }
-    const uint32_t T = prefix;          // the k-th largest key
-    const int need_eq = remaining;      // keys == T to take (>= 1)
+    __syncthreads();
 
-    // ---- emit, deterministic and in position order --------------------------
-    // Warp w owns the contiguous segment [w*seg, (w+1)*seg).  Pass A counts its
-    // keys > T and == T; a block scan turns the counts into offsets; pass B
-    // writes every key > T and the first need_eq keys == T (lowest positions).
-    const int lane = tid & 31, warp = tid >> 5;
+    // ---- the need_eq = remaining lowest positions among the keys equal to T ------
+    if (n_eq == remaining) {
+        for (int w = tid; w < words; w += kThreads) bitmap[w] |= eqmap[w];
+    } else {
+        const int wpt = (words + kThreads - 1) / kThreads;
+        const int w0 = min(words, tid * wpt), w1 = min(words, w0 + wpt);
+        int c = 0;
+        for (int w = w0; w < w1; ++w) c += __popc(eqmap[w]);
+        int total;
+        int before = block_excl_scan(c, sh, &total);
+        for (int w = w0; w < w1 && before < remaining; ++w) {
+            uint32_t e = eqmap[w];
+            const int pc = __popc(e);
+            if (before + pc > remaining) {          // keep only the lowest bits
+                for (int drop = before + pc - remaining; drop > 0; --drop)
+                    e &= ~(0x80000000u >> __clz(e));
+            }
+            bitmap[w] |= e;
+            before += pc;
+        }
+    }
+    __syncthreads();
+
+    // ---- 4. ascending output -------------------------------------------------------
+    bitmap_to_list(sh, bitmap, words, out);
+}
+
+// Rows longer than the bitmap capacity: three radix passes over the whole row, then
+// an ordered two-sweep emission (warp w owns a contiguous segment; one sweep counts,
+// the second writes).
+__global__ void __launch_bounds__(kThreads, 1)
+topk_long_kernel(const float* __restrict__ logits, long long ld, BatchView bv, int k,
+                 int* __restrict__ idx, int* check, int stage_cap) {
+    extern __shared__ __align__(16) uint8_t dyn[];
+    int* hist = reinterpret_cast<int*>(dyn);                                // [4][2048]
+    uint32_t* skeys = reinterpret_cast<uint32_t*>(dyn + kCopies * 2048 * 4);
+    __shared__ Shared sh;
+    __shared__ int s_gt[kWarps], s_eq[kWarps];
+
+    const int t = blockIdx.x, tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    int* out = idx + (long long)t * k;
+    const RowInfo ri = row_info(bv, t, check);
+    if (!ri.ok) {
+        for (int i = tid; i < k; i += kThreads) out[i] = -1;
+        return;
+    }
+    const int n = ri.pos + 1;
+    if (n <= k) {
+        for (int i = tid; i < k; i += kThreads) out[i] = i < n ? i : -1;
+        return;
+    }
+    const float* grow = logits + (long long)t * ld;
+    const Row row{grow, skeys, stage_cap};
+    for (int i = tid; i < kCopies * 2048; i += kThreads) hist[i] = 0;
+    __syncthreads();
+    stage_and_histogram(grow, n, skeys, stage_cap, hist);
+    __syncthreads();
+    int n_def, cnt;
+    const uint32_t b1 = (uint32_t)find_bin(sh, hist, kCopies, 2048, k, &n_def, &cnt);
+    int remaining = k - n_def;
+    uint32_t prefix = b1 << (32 - kTopBits), pmask = ~kLowMask;
+    refine(sh, hist, n, row, 10, 11, prefix, pmask, remaining, &cnt);
+    refine(sh, hist, n, row, 0, 10, prefix, pmask, remaining, &cnt);
+    const uint32_t T = prefix;
+    const int need_eq = remaining;
+
     const int seg = ((n + kWarps - 1) / kWarps + 31) & ~31;
     const int w0 = min(n, warp * seg), w1 = min(n, w0 + seg);
     int c_gt = 0, c_eq = 0;
@@ -150,7 +394,6 @@ topk_kernel(const float* __restrict__ logits, long long ld, BatchView bv, int k,
         c_gt += __popc(__ballot_sync(0xffffffffu, i < w1 && key > T));
         c_eq += __popc(__ballot_sync(0xffffffffu, i < w1 && key == T));
     }
-    __shared__ int s_gt[kWarps], s_eq[kWarps];
     if (lane == 0) {
         s_gt[warp] = c_gt;
         s_eq[warp] = c_eq;
@@ -161,7 +404,7 @@ topk_kernel(const float* __restrict__ logits, long long ld, BatchView bv, int k,
         gt_before += s_gt[v];
         eq_before += s_eq[v];
     }
-    int taken = gt_before + min(eq_before, need_eq);   // output slot of the next taken key
+    int taken = gt_before + min(eq_before, need_eq);
     int eq_seen = eq_before;
     for (int i0 = w0; i0 < w1; i0 += 32) {
         const int i = i0 + lane;
@@ -182,12 +425,26 @@ topk_kernel(const float* __restrict__ logits, long long ld, BatchView bv, int k,
 
 cudaError_t launch_topk(const float* logits, long long ld, const BatchView& bv, int k, int* idx,
                         int* check, cudaStream_t st) {
-    const int staged = bv.max_seq_len < kSmemKeys ? bv.max_seq_len : kSmemKeys;
-    const size_t smem = (size_t)staged * sizeof(uint32_t);
-    cudaError_t e = cudaFuncSetAttribute(topk_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         (int)smem);
-    if (e != cudaSuccess) return e;
-    topk_kernel<<<bv.total_q, kThreads, smem, st>>>(logits, ld, bv, k, idx, check, staged);
+    const int hist_bytes = kCopies * 2048 * 4;
+    const int words = ((bv.max_seq_len + 31) / 32 + 3) & ~3;
+    if (words <= kMaxWords) {
+        const int fixed = hist_bytes + kCandCap * 8 + 2 * words * 4;
+        int stage = (kSmemLimit - kStaticReserve - fixed) / 4 & ~3;
+        if (stage > bv.max_seq_len) stage = bv.max_seq_len;
+        const size_t smem = (size_t)fixed + (size_t)stage * 4;
+        cudaError_t e = cudaFuncSetAttribute(topk_kernel,
+                                             cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+        if (e != cudaSuccess) return e;
+        topk_kernel<<<bv.total_q, kThreads, smem, st>>>(logits, ld, bv, k, idx, check, words,
+                                                        stage);
+    } else {
+        const int stage = (kSmemLimit - kStaticReserve - hist_bytes) / 4 & ~3;
+        const size_t smem = (size_t)hist_bytes + (size_t)stage * 4;
+        cudaError_t e = cudaFuncSetAttribute(topk_long_kernel,
+                                             cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+        if (e != cudaSuccess) return e;
+        topk_long_kernel<<<bv.total_q, kThreads, smem, st>>>(logits, ld, bv, k, idx, check, stage);
+    }
     return cudaGetLastError();
 }
 

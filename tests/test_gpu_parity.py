@@ -116,7 +116,9 @@ def test_small_k_and_fp32_mla_split():
 @pytest.mark.parametrize("n,k,kind", [(5000, 2048, "equal"), (5000, 2048, "three"),
                                       (2049, 2048, "zeros"), (70000, 2048, "three"),
                                       (70000, 2048, "normal"), (2048, 2048, "normal"),
-                                      (100000, 4096, "equal")])
+                                      (100000, 4096, "equal"), (50000, 2048, "coarse"),
+                                      (20000, 2048, "normal"), (9000, 100, "coarse"),
+                                      (300000, 2048, "normal"), (300000, 2048, "three")])
 def test_topk_ties_and_long_rows(n, k, kind):
     g = torch.Generator(device="cuda").manual_seed(n + k)
     if kind == "equal":
@@ -126,6 +128,8 @@ def test_topk_ties_and_long_rows(n, k, kind):
     elif kind == "zeros":  # +0.0 and -0.0 compare equal
         row = torch.zeros(1, n, device="cuda")
         row[0, ::2] = -0.0
+    elif kind == "coarse":  # many exact ties around the k-th score
+        row = torch.round(torch.randn(1, n, generator=g, device="cuda") * 50) / 50
     else:
         row = torch.randn(1, n, generator=g, device="cuda")
     ld = (n + 3) // 4 * 4
