@@ -18,19 +18,23 @@
 //
 // Roles (352 threads): warps 0-3 = softmax (thread = head = TMEM lane), warps 4-9 =
 // gather (3 threads per selected row), warp 10 = TMEM owner and MMA issuer.  The
-// gather is software-pipelined over tiles, per thread: the index of tile j+4, the
-// slot of tile j+3, an L2 bulk prefetch of the rows of tile j+2 and the register
-// loads of tile j+1 are all in flight while tile j is written to shared memory.  The MMAs run on fp16 operands: e4m3 and bf16 values
-// convert to fp16 exactly (bf16 magnitudes above 65504 saturate), and P keeps 11
-// significant bits.
+// gather runs a per-thread pipeline over tiles: the index of tile j+5, the slot of
+// tile j+4 and an L2 prefetch of the rows of tile j+2 are in flight while tile j is
+// copied.  bf16 rows go to shared memory by asynchronous 16-byte copies (no register
+// staging); e4m3 rows are loaded one tile ahead into registers and converted to bf16
+// (exact).  The MMAs take bf16 operands.  P is split as P_hi = bf16(p) and
+// P_lo = bf16(p - P_hi), so that P.V runs as two bf16 products and keeps ~16
+// significant bits of p (bf16 P alone loses up to 2^-9 relative per term, too much
+// for rows dominated by a few large values).
 //
-// Tensor memory: O_v (256 columns), S (64), P (32 = 64 fp16) and query dims 0..319
-// (160 columns); dims 320..575 of the query sit in shared memory next to a 2-stage
-// ring of gathered 64-row tiles (72 KB each, 128-byte swizzled K-major regions of
-// 64 dims).  Per tile: 36 MMAs (M=128, N=64, K=16) for S -- A from TMEM or shared
-// memory -- and 4 MMAs (M=128, N=256, K=16) for P.V_v with A = P in TMEM.  Online
-// softmax in base 2 with lazy rescaling (O and l are rescaled only when the running
-// max grows by more than 2^8).
+// Tensor memory: O_v (256 columns), two 64-column score buffers (S_j in fp32, then
+// P_j = P_hi | P_lo written over it, so S_{j+1} never waits for the softmax of tile
+// j) and query dims 0..255 (128 columns); dims 256..575 of the query sit in shared memory
+// next to a 2-stage ring of gathered 64-row tiles (72 KB each, 128-byte swizzled
+// K-major regions of 64 dims).  Per tile: 36 MMAs (M=128, N=64, K=16) for S -- A
+// from TMEM or shared memory -- and 8 MMAs (M=128, N=256, K=16) for P.V_v with A =
+// P_hi / P_lo in TMEM.  Online softmax in base 2 with lazy rescaling (O and l are
+// rescaled only when the running max grows by more than 2^8).
 #include <climits>
 
 #include "kernels.h"
@@ -45,29 +49,32 @@ constexpr int kHeads = 128;
 constexpr int kTile = 64;
 constexpr int kThreads = 352;
 constexpr int kGatherWarp0 = 4;
-constexpr int kGatherThreads = 192;    // 3 per row of a 64-row tile
+constexpr int kGatherThreads = 192;    // two groups of 96, one per KV stage
+constexpr int kGroupThreads = 96;
 constexpr int kMmaWarp = 10;
 
 constexpr int kStages = 2;
 constexpr int kRegions = 9;                              // 64-dim regions of a 576-dim row
-constexpr uint32_t kQsRegions = 4;                       // query dims 320..575 in smem
+constexpr uint32_t kQsRegions = 5;                       // query dims 256..575 in smem
 constexpr uint32_t kQsBytes = kQsRegions * 16384;        // 128 rows x 128 B per region
 constexpr uint32_t kStageBytes = kRegions * 8192;        // 64 rows x 128 B per region
 constexpr uint32_t kOffQs = 0;
 constexpr uint32_t kOffKV = kOffQs + kQsBytes;
 constexpr uint32_t kOffFlag = kOffKV + kStages * kStageBytes;   // [stage][64] validity bytes
 constexpr uint32_t kOffScale = kOffFlag + kStages * 64;         // [stage][64] fp32 kv scale
-constexpr uint32_t kOffBar = kOffScale + kStages * 256;
+constexpr uint32_t kOffSlot = kOffScale + kStages * 256;       // [stage][64] int slot
+constexpr uint32_t kOffBar = kOffSlot + kStages * 256;
 constexpr uint32_t kNumBars = 12;
 constexpr uint32_t kSmemBytes = kOffBar + kNumBars * 8 + 16 + 1024;
 static_assert(kSmemBytes <= 232448, "shared memory budget");
 
 constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kColO = 0;      // 256 output columns
-constexpr uint32_t kColS = 256;    // 64 score columns
-constexpr uint32_t kColP = 320;    // 32 columns = 64 fp16 probabilities
-constexpr uint32_t kColQ = 352;    // 160 columns = query dims 0..319 as fp16 pairs
-constexpr int kQtSteps = 20;       // K-steps of 16 dims with A in TMEM
+constexpr uint32_t kColS = 256;    // two 64-column buffers: S_j (fp32), then P_j over it
+                                   // (32 columns of bf16 P_hi, 32 of bf16 P_lo)
+constexpr uint32_t kColQ = 384;    // 128 columns = query dims 0..255 as bf16 pairs
+constexpr int kQtSteps = 16;       // K-steps of 16 dims with A in TMEM
+constexpr int kQtChunks = 32;      // 16-byte query chunks held in TMEM
 
 struct Params {
     const uint4* q;            // bf16 [T][128][576] as 16-byte chunks (72 per head)
@@ -100,32 +107,31 @@ __device__ __forceinline__ uint4 ldg16(const void* p) {
     return v;
 }
 
+__device__ __forceinline__ void group_sync(int id, int threads) {
+    asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(threads) : "memory");
+}
+
 __device__ __forceinline__ void sts16(uint32_t saddr, uint4 v) {
     asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};"
                  ::"r"(saddr), "r"(v.x), "r"(v.y), "r"(v.z), "r"(v.w) : "memory");
 }
 
-// Two e4m3 codes (low byte first) -> two fp16 (exact: every e4m3 value is an fp16).
-__device__ __forceinline__ uint32_t e4m3x2_to_f16x2(uint32_t two) {
+// Two e4m3 codes (low byte first) -> two bf16 (exact: every e4m3 value is a bf16;
+// the hardware conversion goes through fp16, which also holds every e4m3 value).
+__device__ __forceinline__ uint32_t e4m3x2_to_bf16x2(uint32_t two) {
     const __half2_raw h = __nv_cvt_fp8x2_to_halfraw2((__nv_fp8x2_storage_t)two, __NV_E4M3);
-    return (uint32_t)h.x | ((uint32_t)h.y << 16);
+    const float2 f = __half22float2(*reinterpret_cast<const __half2*>(&h));
+    const __nv_bfloat162 b = __floats2bfloat162_rn(f.x, f.y);
+    return *reinterpret_cast<const uint32_t*>(&b);
 }
 
-// Two floats -> fp16x2 (lo in the low half), round to nearest, saturating at 65504.
-__device__ __forceinline__ uint32_t pack_f16(float lo, float hi) {
-    uint32_t r;
-    asm("cvt.rn.satfinite.f16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(hi), "f"(lo));
-    return r;
+// 16-byte asynchronous copy global -> shared; src_bytes = 0 writes zeros.
+__device__ __forceinline__ void cp_async16(uint32_t saddr, const void* gptr, uint32_t src_bytes) {
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;"
+                 ::"r"(saddr), "l"(gptr), "r"(src_bytes) : "memory");
 }
-
-// Two bf16 (one 32-bit word) -> two fp16; exact for magnitudes in [2^-14, 65504].
-__device__ __forceinline__ uint32_t bf16x2_to_f16x2(uint32_t v) {
-    return pack_f16(__uint_as_float(v << 16), __uint_as_float(v & 0xFFFF0000u));
-}
-
-__device__ __forceinline__ uint4 bf16x8_to_f16x8(uint4 a) {
-    return make_uint4(bf16x2_to_f16x2(a.x), bf16x2_to_f16x2(a.y), bf16x2_to_f16x2(a.z),
-                      bf16x2_to_f16x2(a.w));
+__device__ __forceinline__ void cp_async_commit_wait_all() {
+    asm volatile("cp.async.commit_group;\n\tcp.async.wait_group 0;" ::: "memory");
 }
 
 __device__ __forceinline__ float fast_exp2(float x) {
@@ -151,11 +157,10 @@ mla_tc_kernel(const Params p) {
     uint64_t* bars = reinterpret_cast<uint64_t*>(base + kOffBar);
     uint64_t* kvfull = bars + 0;    // [2] gather -> MMA / softmax     (192 arrivals)
     uint64_t* kvempty = bars + 2;   // [2] PV done -> gather           (commit)
-    uint64_t* sfull = bars + 4;     // scores ready                    (commit)
-    uint64_t* sempty = bars + 5;    // scores read                     (128)
-    uint64_t* pfull = bars + 6;     // P (and any O rescale) ready     (128)
-    uint64_t* pvdone = bars + 7;    // PV finished                     (commit)
-    uint64_t* qfull = bars + 8;     // query in TMEM + shared memory   (128)
+    uint64_t* sfull = bars + 4;     // [2] S_j ready in buffer j%2     (commit)
+    uint64_t* pfull = bars + 6;     // [2] P_j (and any O rescale) ready (128)
+    uint64_t* pvdone = bars + 8;    // [2] P_j.V finished; buffer j%2 free (commit)
+    uint64_t* qfull = bars + 10;    // query in TMEM + shared memory   (128)
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + kNumBars);
 
     const int warp = threadIdx.x >> 5;
@@ -169,13 +174,14 @@ mla_tc_kernel(const Params p) {
     if (threadIdx.x == 0) {
         s_skip = timed_out_before(p.check) ? 1 : 0;
         for (int i = 0; i < kStages; ++i) {
-            mbar_init(&kvfull[i], kGatherThreads);
+            mbar_init(&kvfull[i], kGroupThreads);
             mbar_init(&kvempty[i], 1);
         }
-        mbar_init(sfull, 1);
-        mbar_init(sempty, 128);
-        mbar_init(pfull, 128);
-        mbar_init(pvdone, 1);
+        for (int i = 0; i < 2; ++i) {
+            mbar_init(&sfull[i], 1);
+            mbar_init(&pfull[i], 128);
+            mbar_init(&pvdone[i], 1);
+        }
         mbar_init(qfull, 128);
         fence_barrier_init();
     }
@@ -191,19 +197,20 @@ mla_tc_kernel(const Params p) {
 
     if (warp >= kGatherWarp0 && warp < kMmaWarp) {
         // ============================================================ gather
+        // Group g (warps 4-6 or 7-9) fills KV stage g with tiles g, g+2, g+4, ...:
+        // the two groups' copies of consecutive tiles overlap.  Thread r < 64 of a
+        // group owns row r: it runs the index -> slot pipeline for the group's
+        // upcoming tiles and publishes the tile's slots in shared memory; then every
+        // warp copies whole 128-byte lines (8 lanes per line, 4 rows per instruction).
         const int gt = threadIdx.x - kGatherWarp0 * 32;     // 0..191
-        const int c = gt / 3, part = gt % 3;                // row of the tile, third of the row
-        constexpr int kN = kFp8 ? 12 : 24;                  // 16-byte loads per thread per tile
+        const int grp = gt / kGroupThreads, gl = gt % kGroupThreads;
+        const int gw = gl >> 5, lane = gl & 31;
         constexpr int kRowBytes = kFp8 ? 576 : 1152;
+        int* srow = reinterpret_cast<int*>(base + kOffSlot) + grp * 64;
         const long long seq_base = (long long)ri.b * p.st_stride;
-        // Per-thread pipeline state for its row c of upcoming tiles: no load result is
-        // consumed in the iteration that issues the load.
-        int idx5 = -1;                                  // index of tile j+5
-        int raw_s4 = -1;                                // slot-table entry of tile j+4 (unchecked)
-        long long slot1 = -1, slot2 = -1, slot3 = -1;   // checked slots of tiles j+1..j+3
         auto fetch_idx = [&](int j) -> int {
-            const int i = i0 + j * kTile + c;
-            return (j < n_tiles && i < i1) ? __ldg(p.idx + (long long)t * p.k + i) : -1;
+            const int i = i0 + j * kTile + gl;
+            return (gl < kTile && j < n_tiles && i < i1) ? __ldg(p.idx + (long long)t * p.k + i) : -1;
         };
         // Slot-table entry for index s, or a sentinel for a skipped entry / an index
         // past the query position (table entries are checked separately).
@@ -213,125 +220,144 @@ mla_tc_kernel(const Params p) {
             if (s > ri.pos) return kPastPos;
             return __ldg(p.slot_table + seq_base + s);
         };
-        auto check_slot = [&](int raw) -> long long {   // -1 for skipped / bad entries
+        auto check_slot = [&](int raw) -> int {   // -1 for skipped / bad entries
             if (raw == kSkip) return -1;
             if (raw == kPastPos || raw < 0 || (long long)raw >= p.num_slots) {
-                if (part == 0) report(p.check, raw == kPastPos ? kCheckBadIndex : kCheckBadPage);
+                report(p.check, raw == kPastPos ? kCheckBadIndex : kCheckBadPage);
                 return -1;
             }
             return raw;
         };
-        auto prefetch_row = [&](long long sl) {
-            if (sl >= 0)
-                asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;"
-                             ::"l"(p.kv + sl * kRowBytes + part * kN * 16), "r"(kN * 16) : "memory");
-        };
-        uint4 v[kN];
-        float scale = 1.0f;
-        auto load_regs = [&](long long sl) {
-            const uint4* row = reinterpret_cast<const uint4*>(p.kv + (sl < 0 ? 0 : sl) * kRowBytes) + part * kN;
-#pragma unroll
-            for (int u = 0; u < kN; ++u) v[u] = sl >= 0 ? ldg16(row + u) : make_uint4(0, 0, 0, 0);
-            scale = (sl >= 0 && kFp8 && p.kv_scale) ? __ldg(p.kv_scale + sl) : 1.0f;
-        };
-        // prologue: tiles 0..4 in flight
-        long long slot0 = -1;
-        if (n_tiles > 0) {
-            const int x0 = fetch_idx(0), x1 = fetch_idx(1), x2 = fetch_idx(2), x3 = fetch_idx(3),
-                      x4 = fetch_idx(4);
-            idx5 = fetch_idx(5);
-            const int r0 = fetch_slot(x0), r1 = fetch_slot(x1), r2 = fetch_slot(x2),
-                      r3 = fetch_slot(x3);
-            raw_s4 = fetch_slot(x4);
-            slot0 = check_slot(r0);
-            slot1 = check_slot(r1);
-            slot2 = check_slot(r2);
-            slot3 = check_slot(r3);
-            prefetch_row(slot1);
-            load_regs(slot0);
+        // pipeline over the group's own tiles: slots of tiles j and j+2, the table
+        // entry of tile j+4 and the index of tile j+6 are in flight at tile j
+        int sl_cur = -1, sl_next = -1, raw_n2 = kSkip, idx_n3 = -1;
+        if (grp < n_tiles) {
+            const int x0 = fetch_idx(grp), x1 = fetch_idx(grp + 2), x2 = fetch_idx(grp + 4);
+            idx_n3 = fetch_idx(grp + 6);
+            const int r0 = fetch_slot(x0), r1 = fetch_slot(x1);
+            raw_n2 = fetch_slot(x2);
+            sl_cur = check_slot(r0);
+            sl_next = check_slot(r1);
         }
-        long long cur = slot0;                          // slot of the tile held in v
-        for (int j = 0; j < n_tiles; ++j) {
-            const int stage = j % kStages;
+        const int stage = grp;
+        const uint32_t st = sb + kOffKV + stage * kStageBytes;
+        for (int j = grp; j < n_tiles; j += kStages) {
+            if (sl_next >= 0)
+                asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;"
+                             ::"l"(p.kv + (long long)sl_next * kRowBytes), "r"(kRowBytes) : "memory");
             if (!mbar_wait_warp(&kvempty[stage], ((j / kStages) & 1) ^ 1, p.check)) break;
-            const uint32_t st = sb + kOffKV + stage * kStageBytes;
-            if constexpr (kFp8) {
-#pragma unroll
-                for (int u = 0; u < kN; ++u) {
-                    const int g = 2 * (part * kN + u);      // first of the two fp16 chunks
-                    const uint4 a = v[u];
-                    const uint4 lo = make_uint4(e4m3x2_to_f16x2(a.x & 0xFFFF), e4m3x2_to_f16x2(a.x >> 16),
-                                                e4m3x2_to_f16x2(a.y & 0xFFFF), e4m3x2_to_f16x2(a.y >> 16));
-                    const uint4 hi = make_uint4(e4m3x2_to_f16x2(a.z & 0xFFFF), e4m3x2_to_f16x2(a.z >> 16),
-                                                e4m3x2_to_f16x2(a.w & 0xFFFF), e4m3x2_to_f16x2(a.w >> 16));
-                    sts16(st + (g >> 3) * 8192 + sw128(c, g & 7), lo);
-                    sts16(st + ((g + 1) >> 3) * 8192 + sw128(c, (g + 1) & 7), hi);
+            if (gl < kTile) {
+                srow[gl] = sl_cur;
+                vflag[stage * 64 + gl] = sl_cur >= 0 ? 1 : 0;
+                colscale[stage * 64 + gl] =
+                    (kFp8 && sl_cur >= 0 && p.kv_scale) ? __ldg(p.kv_scale + sl_cur) : 1.0f;
+            }
+            group_sync(1 + grp, kGroupThreads);
+            if constexpr (!kFp8) {
+                // 64 rows x 9 regions of 128 bytes = 144 units of 4 rows; warp gw takes
+                // units gw, gw+3, ...; a skipped or bad row becomes zeros (score masked)
+                const int chunk = lane & 7;
+#pragma unroll 8
+                for (int u = gw; u < 144; u += 3) {
+                    const int rg = u / 9, region = u - rg * 9;
+                    const int row = 4 * rg + (lane >> 3);
+                    const int sl = srow[row];
+                    const uint8_t* src = p.kv + (long long)(sl < 0 ? 0 : sl) * 1152 + region * 128 + chunk * 16;
+                    cp_async16(st + region * 8192 + sw128(row, chunk), src, sl >= 0 ? 16u : 0u);
                 }
             } else {
+                // 64 rows x 36 pieces of 16 e4m3 codes; thread gl takes pieces gl + 96 i
+                uint4 v[24];
 #pragma unroll
-                for (int u = 0; u < kN; ++u) {
-                    const int g = part * kN + u;
-                    sts16(st + (g >> 3) * 8192 + sw128(c, g & 7), bf16x8_to_f16x8(v[u]));
+                for (int i = 0; i < 24; ++i) {
+                    const int q = gl + kGroupThreads * i, row = q / 36, pc = q - row * 36;
+                    const int sl = srow[row];
+                    v[i] = sl >= 0 ? ldg16(p.kv + (long long)sl * 576 + pc * 16) : make_uint4(0, 0, 0, 0);
+                }
+#pragma unroll
+                for (int i = 0; i < 24; ++i) {
+                    const int q = gl + kGroupThreads * i, row = q / 36, pc = q - row * 36;
+                    const int g = 2 * pc;                       // first of the two bf16 chunks
+                    const uint4 a = v[i];
+                    const uint4 lo = make_uint4(e4m3x2_to_bf16x2(a.x & 0xFFFF), e4m3x2_to_bf16x2(a.x >> 16),
+                                                e4m3x2_to_bf16x2(a.y & 0xFFFF), e4m3x2_to_bf16x2(a.y >> 16));
+                    const uint4 hi = make_uint4(e4m3x2_to_bf16x2(a.z & 0xFFFF), e4m3x2_to_bf16x2(a.z >> 16),
+                                                e4m3x2_to_bf16x2(a.w & 0xFFFF), e4m3x2_to_bf16x2(a.w >> 16));
+                    sts16(st + (g >> 3) * 8192 + sw128(row, g & 7), lo);
+                    sts16(st + ((g + 1) >> 3) * 8192 + sw128(row, (g + 1) & 7), hi);
                 }
             }
-            if (part == 0) {
-                vflag[stage * 64 + c] = cur >= 0 ? 1 : 0;
-                colscale[stage * 64 + c] = scale;
-            }
+            // advance the pipeline (independent loads, issued before waiting on the copies)
+            const int nxt = check_slot(raw_n2);     // loaded one round ago
+            raw_n2 = fetch_slot(idx_n3);             // index loaded one round ago
+            idx_n3 = fetch_idx(j + 8);
+            if constexpr (!kFp8) cp_async_commit_wait_all();
             fence_proxy_async_smem();
             mbar_arrive(&kvfull[stage]);
-            // advance the pipeline by one tile
-            if (j + 1 < n_tiles) load_regs(slot1);
-            prefetch_row(slot2);
-            const long long s4 = check_slot(raw_s4);   // loaded one iteration ago
-            raw_s4 = fetch_slot(idx5);                  // index loaded one iteration ago
-            idx5 = fetch_idx(j + 6);
-            cur = slot1;
-            slot1 = slot2;
-            slot2 = slot3;
-            slot3 = s4;
+            sl_cur = sl_next;
+            sl_next = nxt;
         }
     } else if (warp == kMmaWarp) {
         // ============================================================ MMA issuer
         if (elect_one() && n_tiles > 0) {
             bool alive = mbar_wait(qfull, 0, p.check);
             tc_fence_after();
-            const uint32_t idesc_qk = instr_desc(0, 0, 0, 0, kTile, kHeads);   // fp16 x fp16
-            const uint32_t idesc_pv = instr_desc(0, 0, 0, 1, 256, kHeads);
+            const uint32_t idesc_qk = instr_desc(1, 1, 0, 0, kTile, kHeads);   // bf16 x bf16
+            const uint32_t idesc_pv = instr_desc(1, 1, 0, 1, 256, kHeads);
             const uint32_t qs = sb + kOffQs;
-            for (int j = 0; alive && j <= n_tiles; ++j) {
-                if (j < n_tiles) {
-                    const int stage = j % kStages;
-                    if (!mbar_wait(&kvfull[stage], (j / kStages) & 1, p.check)) break;
-                    if (j >= 1 && !mbar_wait(sempty, (j - 1) & 1, p.check)) break;
-                    tc_fence_after();
-                    const uint32_t kva = sb + kOffKV + stage * kStageBytes;
+            // S_j = Q . KV_j^T (36 K-steps of 16: dims 0..255 with A in TMEM, the rest
+            // with A in shared memory)
+            auto issue_qk = [&](int jt) {
+                const uint32_t kva = sb + kOffKV + (jt % kStages) * kStageBytes;
+                const uint32_t sbuf = tmem + kColS + 64 * (jt & 1);
 #pragma unroll
-                    for (int s = 0; s < 36; ++s) {
-                        const uint64_t bdesc =
-                            smem_desc(kva + (s >> 2) * 8192 + (s & 3) * 32, 16, 1024, kLayoutSw128);
-                        if (s < kQtSteps)
-                            mma_f16_ts(tmem + kColS, tmem + kColQ + 8 * s, bdesc, idesc_qk, s > 0 ? 1u : 0u);
-                        else
-                            mma_f16(tmem + kColS,
-                                    smem_desc(qs + ((s - kQtSteps) >> 2) * 16384 + (s & 3) * 32, 16, 1024,
-                                              kLayoutSw128),
-                                    bdesc, idesc_qk, 1u);
-                    }
-                    mma_commit(sfull);
+                for (int s = 0; s < 36; ++s) {
+                    const uint64_t bdesc =
+                        smem_desc(kva + (s >> 2) * 8192 + (s & 3) * 32, 16, 1024, kLayoutSw128);
+                    if (s < kQtSteps)
+                        mma_f16_ts(sbuf, tmem + kColQ + 8 * s, bdesc, idesc_qk, s > 0 ? 1u : 0u);
+                    else
+                        mma_f16(sbuf,
+                                smem_desc(qs + ((s - kQtSteps) >> 2) * 16384 + (s & 3) * 32, 16, 1024,
+                                          kLayoutSw128),
+                                bdesc, idesc_qk, 1u);
                 }
-                if (j >= 1) {
-                    const int jj = j - 1, stage = jj % kStages;
-                    if (!mbar_wait(pfull, jj & 1, p.check)) break;
-                    tc_fence_after();
-                    const uint32_t va = sb + kOffKV + stage * kStageBytes + vh * 4 * 8192;
+                mma_commit(&sfull[jt & 1]);
+            };
+            // O_v += P_hi . V_v + P_lo . V_v (P = P_hi + P_lo to ~16 significant bits)
+            auto issue_pv = [&](int jt) {
+                const int stage = jt % kStages;
+                const uint32_t va = sb + kOffKV + stage * kStageBytes + vh * 4 * 8192;
 #pragma unroll
-                    for (int kk = 0; kk < 4; ++kk)
-                        mma_f16_ts(tmem + kColO, tmem + kColP + 8 * kk,
-                                   smem_desc(va + kk * 2048, 8192, 1024, kLayoutSw128), idesc_pv,
-                                   (jj > 0 || kk > 0) ? 1u : 0u);
-                    mma_commit(&kvempty[stage]);
-                    mma_commit(pvdone);
+                for (int kk = 0; kk < 8; ++kk)
+                    mma_f16_ts(tmem + kColO, tmem + kColS + 64 * (jt & 1) + (kk < 4 ? 0 : 32) + 8 * (kk & 3),
+                               smem_desc(va + (kk & 3) * 2048, 8192, 1024, kLayoutSw128), idesc_pv,
+                               (jt > 0 || kk > 0) ? 1u : 0u);
+                mma_commit(&kvempty[stage]);
+                mma_commit(&pvdone[jt & 1]);
+            };
+            // Round j issues S_j and P_{j-1}.V in whichever order their inputs arrive
+            // (P.V first when both are ready: it frees a KV stage for the gather).
+            // S_j reuses buffer j%2 once P_{j-2}.V has read the P stored there.
+            for (int j = 0; alive && j <= n_tiles; ++j) {
+                bool qk = j < n_tiles, pv = j >= 1;
+                const uint32_t kv_par = (j / kStages) & 1;
+                const long long t0 = clock64();
+                while (qk || pv) {
+                    if (pv && mbar_test(&pfull[(j - 1) & 1], ((j - 1) >> 1) & 1)) {
+                        tc_fence_after();
+                        issue_pv(j - 1);
+                        pv = false;
+                    } else if (qk && mbar_test(&kvfull[j % kStages], kv_par) &&
+                               (j < 2 || mbar_test(&pvdone[j & 1], ((j - 2) >> 1) & 1))) {
+                        tc_fence_after();
+                        issue_qk(j);
+                        qk = false;
+                    } else if (clock64() - t0 > kWaitLimitCycles) {
+                        report(p.check, kCheckTimeout);
+                        alive = false;
+                        break;
+                    }
                 }
             }
         }
@@ -339,7 +365,7 @@ mla_tc_kernel(const Params p) {
         // ============================================================ softmax
         const int h = threadIdx.x;                       // head == TMEM lane
         const uint32_t lane_base = tmem + ((uint32_t)(warp * 32) << 16);
-        {   // query row h: dims 0..319 into TMEM as fp16 pairs, 320..575 into smem
+        {   // query row h: dims 0..255 into TMEM as bf16 pairs, 256..575 into smem
             const uint4* qrow = p.q + ((long long)t * kHeads + h) * 72;
             if (ri.ok) asm volatile("cp.async.bulk.prefetch.L2.global [%0], 1152;" ::"l"(qrow) : "memory");
 #pragma unroll
@@ -350,11 +376,11 @@ mla_tc_kernel(const Params p) {
 #pragma unroll
                 for (int g = 0; g < 24; g += 2) {
                     const int gg = g0 + g;
-                    const uint4 a = bf16x8_to_f16x8(qv[g]), b = bf16x8_to_f16x8(qv[g + 1]);
-                    if (gg < 40) {
+                    const uint4 a = qv[g], b = qv[g + 1];
+                    if (gg < kQtChunks) {
                         tmem_st8(lane_base + kColQ + 4 * gg, a.x, a.y, a.z, a.w, b.x, b.y, b.z, b.w);
                     } else {
-                        const int c0 = gg - 40;              // chunk index within dims 320..575
+                        const int c0 = gg - kQtChunks;       // chunk index within dims 256..575
                         sts16(sb + kOffQs + (c0 >> 3) * 16384 + sw128(h, c0 & 7), a);
                         sts16(sb + kOffQs + ((c0 + 1) >> 3) * 16384 + sw128(h, (c0 + 1) & 7), b);
                     }
@@ -370,15 +396,14 @@ mla_tc_kernel(const Params p) {
         for (int j = 0; alive && j < n_tiles; ++j) {
             const int stage = j % kStages;
             float x[64];
+            const uint32_t sb_col = kColS + 64 * (j & 1);  // S_j, then P_j
             {   // ---- scores of tile j
-                if (!mbar_wait_warp(sfull, j & 1, p.check)) { alive = false; break; }
+                if (!mbar_wait_warp(&sfull[j & 1], (j >> 1) & 1, p.check)) { alive = false; break; }
                 tc_fence_after();
                 uint32_t a[32], c[32];
-                tmem_ld32(lane_base + kColS, a);
-                tmem_ld32(lane_base + kColS + 32, c);
+                tmem_ld32(lane_base + sb_col, a);
+                tmem_ld32(lane_base + sb_col + 32, c);
                 tmem_ld_wait();
-                tc_fence_before();
-                mbar_arrive(sempty);                       // the next QK may overwrite S
 #pragma unroll
                 for (int i = 0; i < 32; ++i) {
                     x[i] = __uint_as_float(a[i]);
@@ -429,19 +454,22 @@ mla_tc_kernel(const Params p) {
             const bool warp_rescale = __any_sync(0xffffffffu, need) && j > 0;
             const float msub = m_run == -INFINITY ? 0.f : m_run;   // exp2(-inf) = +0
             float ls[4] = {0.f, 0.f, 0.f, 0.f};
-            uint32_t pk[32];
+            uint32_t ph[32], pl[32];
 #pragma unroll
             for (int i = 0; i < 64; i += 2) {
                 const float e0 = fast_exp2(fmaf(x[i], sc, -msub));
                 const float e1 = fast_exp2(fmaf(x[i + 1], sc, -msub));
                 ls[(i >> 1) & 3] += e0 + e1;
-                pk[i / 2] = kFp8 ? pack_f16(e0 * cs[i], e1 * cs[i + 1]) : pack_f16(e0, e1);
+                const float v0 = kFp8 ? e0 * cs[i] : e0, v1 = kFp8 ? e1 * cs[i + 1] : e1;
+                const uint32_t hi = pack_bf16(v0, v1);
+                ph[i / 2] = hi;
+                pl[i / 2] = pack_bf16(v0 - __uint_as_float(hi << 16), v1 - __uint_as_float(hi & 0xFFFF0000u));
             }
             l_run = l_run * alpha + ((ls[0] + ls[1]) + (ls[2] + ls[3]));
-            // ---- P (and O) are free once the previous PV has finished
-            if (j >= 1 && !mbar_wait_warp(pvdone, (j - 1) & 1, p.check)) { alive = false; break; }
-            tc_fence_after();
+            // ---- O may be rescaled only once the previous PV has finished
             if (warp_rescale) {
+                if (!mbar_wait_warp(&pvdone[(j - 1) & 1], ((j - 1) >> 1) & 1, p.check)) { alive = false; break; }
+                tc_fence_after();
 #pragma unroll 1
                 for (int cc = 0; cc < 8; ++cc) {
                     uint32_t o[32];
@@ -452,13 +480,15 @@ mla_tc_kernel(const Params p) {
                     tmem_st32(lane_base + kColO + cc * 32, o);
                 }
             }
-            tmem_st32(lane_base + kColP, pk);
+            tmem_st32(lane_base + sb_col, ph);
+            tmem_st32(lane_base + sb_col + 32, pl);
             tmem_st_wait();
             tc_fence_before();
-            mbar_arrive(pfull);
+            mbar_arrive(&pfull[j & 1]);
         }
         // ---- epilogue: O_v / l and lse
-        const bool have = alive && n_tiles > 0 && mbar_wait_warp(pvdone, (n_tiles - 1) & 1, p.check);
+        const bool have = alive && n_tiles > 0 &&
+                          mbar_wait_warp(&pvdone[(n_tiles - 1) & 1], ((n_tiles - 1) >> 1) & 1, p.check);
         tc_fence_after();
         const float inv = (have && l_run > 0.f) ? 1.0f / l_run : 0.f;
         const float lse_v = (have && l_run > 0.f) ? (m_run + log2f(l_run)) * 0.69314718055994531f
