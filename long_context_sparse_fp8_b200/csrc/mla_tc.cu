@@ -111,6 +111,13 @@ __device__ __forceinline__ void group_sync(int id, int threads) {
     asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(threads) : "memory");
 }
 
+__device__ __forceinline__ uint4 lds16(uint32_t saddr) {
+    uint4 v;
+    asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];"
+                 : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w) : "r"(saddr) : "memory");
+    return v;
+}
+
 __device__ __forceinline__ void sts16(uint32_t saddr, uint4 v) {
     asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};"
                  ::"r"(saddr), "r"(v.x), "r"(v.y), "r"(v.z), "r"(v.w) : "memory");
@@ -147,7 +154,7 @@ __device__ __forceinline__ uint32_t pack_bf16(float a, float b) {
 
 template <bool kFp8>
 __global__ void __launch_bounds__(kThreads, 1)
-mla_tc_kernel(const Params p) {
+mla_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const Params p) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t* base = reinterpret_cast<uint8_t*>(
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -161,6 +168,7 @@ mla_tc_kernel(const Params p) {
     uint64_t* pfull = bars + 6;     // [2] P_j (and any O rescale) ready (128)
     uint64_t* pvdone = bars + 8;    // [2] P_j.V finished; buffer j%2 free (commit)
     uint64_t* qfull = bars + 10;    // query in TMEM + shared memory   (128)
+    uint64_t* qload = bars + 11;    // query tiles landed (TMA bytes)
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + kNumBars);
 
     const int warp = threadIdx.x >> 5;
@@ -183,7 +191,18 @@ mla_tc_kernel(const Params p) {
             mbar_init(&pvdone[i], 1);
         }
         mbar_init(qfull, 128);
+        mbar_init(qload, 1);
         fence_barrier_init();
+        // the query row block [128 heads][576] as nine 64-dim swizzled tiles: dims
+        // 256..575 straight into their shared-memory home, dims 0..255 into KV stage 0
+        // for the softmax threads to move into TMEM
+        if (ri.ok) {
+            prefetch_tmap(&tm_q);
+            mbar_arrive_expect_tx(qload, 9 * 16384);
+            for (int r = 0; r < 9; ++r)
+                tma_load_2d(base + (r < 4 ? kOffKV + r * 16384 : kOffQs + (r - 4) * 16384), &tm_q,
+                            64 * r, t * kHeads, qload);
+        }
     }
     if (warp == kMmaWarp) {
         tmem_alloc(tmem_slot, kTmemCols);
@@ -241,6 +260,7 @@ mla_tc_kernel(const Params p) {
         }
         const int stage = grp;
         const uint32_t st = sb + kOffKV + stage * kStageBytes;
+        if (grp == 0 && n_tiles > 0) mbar_wait_warp(qfull, 0, p.check);   // stage 0 held query tiles
         for (int j = grp; j < n_tiles; j += kStages) {
             if (sl_next >= 0)
                 asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;"
@@ -365,31 +385,22 @@ mla_tc_kernel(const Params p) {
         // ============================================================ softmax
         const int h = threadIdx.x;                       // head == TMEM lane
         const uint32_t lane_base = tmem + ((uint32_t)(warp * 32) << 16);
-        {   // query row h: dims 0..255 into TMEM as bf16 pairs, 256..575 into smem
-            const uint4* qrow = p.q + ((long long)t * kHeads + h) * 72;
-            if (ri.ok) asm volatile("cp.async.bulk.prefetch.L2.global [%0], 1152;" ::"l"(qrow) : "memory");
+        {   // query row h, dims 0..255: from the staging tiles in KV stage 0 into TMEM
+            // (waited for whenever issued: no copy may still be in flight at exit)
+            if (ri.ok) mbar_wait_warp(qload, 0, p.check);
 #pragma unroll
-            for (int g0 = 0; g0 < 72; g0 += 24) {
-                uint4 qv[24];
-#pragma unroll
-                for (int g = 0; g < 24; ++g) qv[g] = ri.ok ? ldg16(qrow + g0 + g) : make_uint4(0, 0, 0, 0);
-#pragma unroll
-                for (int g = 0; g < 24; g += 2) {
-                    const int gg = g0 + g;
-                    const uint4 a = qv[g], b = qv[g + 1];
-                    if (gg < kQtChunks) {
-                        tmem_st8(lane_base + kColQ + 4 * gg, a.x, a.y, a.z, a.w, b.x, b.y, b.z, b.w);
-                    } else {
-                        const int c0 = gg - kQtChunks;       // chunk index within dims 256..575
-                        sts16(sb + kOffQs + (c0 >> 3) * 16384 + sw128(h, c0 & 7), a);
-                        sts16(sb + kOffQs + ((c0 + 1) >> 3) * 16384 + sw128(h, (c0 + 1) & 7), b);
-                    }
+            for (int g = 0; g < kQtChunks; g += 2) {
+                uint4 a = make_uint4(0, 0, 0, 0), b = a;
+                if (ri.ok) {
+                    const uint32_t src = sb + kOffKV + (g >> 3) * 16384;
+                    a = lds16(src + sw128(h, g & 7));
+                    b = lds16(src + sw128(h, (g + 1) & 7));
                 }
+                tmem_st8(lane_base + kColQ + 4 * g, a.x, a.y, a.z, a.w, b.x, b.y, b.z, b.w);
             }
             tmem_st_wait();
-            fence_proxy_async_smem();
             tc_fence_before();
-            mbar_arrive(qfull);
+            mbar_arrive(qfull);                         // also: KV stage 0 may be refilled
         }
         float m_run = -INFINITY, l_run = 0.f;
         bool alive = true;
@@ -564,13 +575,18 @@ cudaError_t launch_mla_tc(const void* q, float scale, const CacheView& kv, const
     p.o_part = o_part;
     p.lse_part = lse_part;
     p.check = check;
+    CUtensorMap tm_q;
+    cudaError_t me = make_tensor_map_2d(&tm_q, q, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, 576,
+                                        (unsigned long long)bv.total_q * kHeads, 1152, 64, kHeads,
+                                        CU_TENSOR_MAP_SWIZZLE_128B);
+    if (me != cudaSuccess) return me;
     const bool fp8 = kv.dtype == kE4M3;
     auto kern = fp8 ? mla_tc_kernel<true> : mla_tc_kernel<false>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          (int)kSmemBytes);
     if (e != cudaSuccess) return e;
     dim3 grid(2 * bv.total_q * nsplit);
-    kern<<<grid, kThreads, kSmemBytes, st>>>(p);
+    kern<<<grid, kThreads, kSmemBytes, st>>>(tm_q, p);
     return cudaGetLastError();
 }
 
