@@ -316,8 +316,13 @@ cudaError_t launch_indexer_fp8_tc(const void* q, const float* q_scale, const flo
     const int G = T <= 2 * bv.num_seqs ? 1 : 4;
     const int groups = (T + G - 1) / G;
     const int tiles_max = (bv.max_seq_len + kTileKeys - 1) / kTileKeys;
-    const int target = 4 * kNumSMs;
+    // About 4 CTAs per SM (2 resident) balance long, uneven rows; when that would
+    // leave fewer than 16 key tiles per CTA, one wave of 2 CTAs per SM is used
+    // instead, so that the per-CTA setup is paid once per SM slot.
+    const int target = 4 * kNumSMs, slots = 2 * kNumSMs;
     int chunks = groups >= target / 2 ? 1 : (target + groups - 1) / groups;
+    if (groups < slots && tiles_max / chunks < 16) chunks = slots / groups;
+    if (chunks < 1) chunks = 1;
     if (chunks > tiles_max) chunks = tiles_max;
     const int C = (tiles_max + chunks - 1) / chunks;
     chunks = (tiles_max + C - 1) / C;

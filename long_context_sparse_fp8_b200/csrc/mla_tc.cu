@@ -22,18 +22,18 @@
 // tile j+4 and an L2 prefetch of the rows of tile j+2 are in flight while tile j is
 // copied.  bf16 rows go to shared memory by asynchronous 16-byte copies (no register
 // staging); e4m3 rows are loaded one tile ahead into registers and converted to bf16
-// (exact).  The MMAs take bf16 operands.  P is split as P_hi = bf16(p) and
-// P_lo = bf16(p - P_hi), so that P.V runs as two bf16 products and keeps ~16
-// significant bits of p (bf16 P alone loses up to 2^-9 relative per term, too much
-// for rows dominated by a few large values).
+// (exact).  S = Q.K^T runs on bf16 operands.  P is kept in fp16 (11 significant
+// bits; bf16 P loses up to 2^-9 relative per term, too much for rows dominated by a
+// few large values), so once S_j has read a tile, the gather group converts this
+// CTA's V columns of it in place from bf16 to fp16 (exact for magnitudes in
+// [2^-14, 65504]; larger ones saturate) while the softmax runs, and P.V runs on fp16.
 //
 // Tensor memory: O_v (256 columns), two 64-column score buffers (S_j in fp32, then
-// P_j = P_hi | P_lo written over it, so S_{j+1} never waits for the softmax of tile
-// j) and query dims 0..255 (128 columns); dims 256..575 of the query sit in shared memory
+// P_j in fp16 written over it, so S_{j+1} never waits for the softmax of tile j) and query dims 0..255 (128 columns); dims 256..575 of the query sit in shared memory
 // next to a 2-stage ring of gathered 64-row tiles (72 KB each, 128-byte swizzled
 // K-major regions of 64 dims).  Per tile: 36 MMAs (M=128, N=64, K=16) for S -- A
-// from TMEM or shared memory -- and 8 MMAs (M=128, N=256, K=16) for P.V_v with A =
-// P_hi / P_lo in TMEM.  Online softmax in base 2 with lazy rescaling (O and l are
+// from TMEM or shared memory -- and 4 MMAs (M=128, N=256, K=16) for P.V_v with A =
+// P in TMEM.  Online softmax in base 2 with lazy rescaling (O and l are
 // rescaled only when the running max grows by more than 2^8).
 #include <climits>
 
@@ -64,14 +64,14 @@ constexpr uint32_t kOffFlag = kOffKV + kStages * kStageBytes;   // [stage][64] v
 constexpr uint32_t kOffScale = kOffFlag + kStages * 64;         // [stage][64] fp32 kv scale
 constexpr uint32_t kOffSlot = kOffScale + kStages * 256;       // [stage][64] int slot
 constexpr uint32_t kOffBar = kOffSlot + kStages * 256;
-constexpr uint32_t kNumBars = 12;
+constexpr uint32_t kNumBars = 16;
 constexpr uint32_t kSmemBytes = kOffBar + kNumBars * 8 + 16 + 1024;
 static_assert(kSmemBytes <= 232448, "shared memory budget");
 
 constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kColO = 0;      // 256 output columns
-constexpr uint32_t kColS = 256;    // two 64-column buffers: S_j (fp32), then P_j over it
-                                   // (32 columns of bf16 P_hi, 32 of bf16 P_lo)
+constexpr uint32_t kColS = 256;    // two 64-column buffers: S_j (fp32), then P_j (fp16,
+                                   // 32 columns) over it
 constexpr uint32_t kColQ = 384;    // 128 columns = query dims 0..255 as bf16 pairs
 constexpr int kQtSteps = 16;       // K-steps of 16 dims with A in TMEM
 constexpr int kQtChunks = 32;      // 16-byte query chunks held in TMEM
@@ -141,6 +141,22 @@ __device__ __forceinline__ void cp_async_commit_wait_all() {
     asm volatile("cp.async.commit_group;\n\tcp.async.wait_group 0;" ::: "memory");
 }
 
+// Two floats -> fp16x2 (lo in the low half), round to nearest, saturating at 65504.
+__device__ __forceinline__ uint32_t pack_f16(float lo, float hi) {
+    uint32_t r;
+    asm("cvt.rn.satfinite.f16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(hi), "f"(lo));
+    return r;
+}
+
+// Eight bf16 -> eight fp16: exact for magnitudes in [2^-14, 65504] (larger ones
+// saturate; smaller ones keep an absolute precision of 2^-24).
+__device__ __forceinline__ uint4 bf16x8_to_f16x8(uint4 a) {
+    auto cv = [](uint32_t v) {
+        return pack_f16(__uint_as_float(v << 16), __uint_as_float(v & 0xFFFF0000u));
+    };
+    return make_uint4(cv(a.x), cv(a.y), cv(a.z), cv(a.w));
+}
+
 __device__ __forceinline__ float fast_exp2(float x) {
     float y;
     asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
@@ -169,6 +185,7 @@ mla_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const Params p) {
     uint64_t* pvdone = bars + 8;    // [2] P_j.V finished; buffer j%2 free (commit)
     uint64_t* qfull = bars + 10;    // query in TMEM + shared memory   (128)
     uint64_t* qload = bars + 11;    // query tiles landed (TMA bytes)
+    uint64_t* vconv = bars + 12;    // [2] V_v of stage s converted to fp16 (96)
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + kNumBars);
 
     const int warp = threadIdx.x >> 5;
@@ -192,6 +209,8 @@ mla_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const Params p) {
         }
         mbar_init(qfull, 128);
         mbar_init(qload, 1);
+        mbar_init(&vconv[0], kGroupThreads);
+        mbar_init(&vconv[1], kGroupThreads);
         fence_barrier_init();
         // the query row block [128 heads][576] as nine 64-dim swizzled tiles: dims
         // 256..575 straight into their shared-memory home, dims 0..255 into KV stage 0
@@ -314,6 +333,18 @@ mla_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const Params p) {
             if constexpr (!kFp8) cp_async_commit_wait_all();
             fence_proxy_async_smem();
             mbar_arrive(&kvfull[stage]);
+            // once S_j has read the bf16 rows, convert this CTA's V columns in place to
+            // fp16 for P.V (P is fp16: bf16 P keeps too few bits, see above)
+            if (!mbar_wait_warp(&sfull[stage], (j >> 1) & 1, p.check)) break;
+            tc_fence_after();
+            const uint32_t vb = st + vh * 4 * 8192;
+#pragma unroll 4
+            for (int q = gl; q < 4 * 512; q += kGroupThreads) {
+                const uint32_t a = vb + q * 16;
+                sts16(a, bf16x8_to_f16x8(lds16(a)));
+            }
+            fence_proxy_async_smem();
+            mbar_arrive(&vconv[stage]);
             sl_cur = sl_next;
             sl_next = nxt;
         }
@@ -323,7 +354,7 @@ mla_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const Params p) {
             bool alive = mbar_wait(qfull, 0, p.check);
             tc_fence_after();
             const uint32_t idesc_qk = instr_desc(1, 1, 0, 0, kTile, kHeads);   // bf16 x bf16
-            const uint32_t idesc_pv = instr_desc(1, 1, 0, 1, 256, kHeads);
+            const uint32_t idesc_pv = instr_desc(0, 0, 0, 1, 256, kHeads);   // fp16 P x fp16 V
             const uint32_t qs = sb + kOffQs;
             // S_j = Q . KV_j^T (36 K-steps of 16: dims 0..255 with A in TMEM, the rest
             // with A in shared memory)
@@ -344,14 +375,14 @@ mla_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const Params p) {
                 }
                 mma_commit(&sfull[jt & 1]);
             };
-            // O_v += P_hi . V_v + P_lo . V_v (P = P_hi + P_lo to ~16 significant bits)
+            // O_v += P . V_v (fp16 operands; K = 64 tokens in four steps of 16)
             auto issue_pv = [&](int jt) {
                 const int stage = jt % kStages;
                 const uint32_t va = sb + kOffKV + stage * kStageBytes + vh * 4 * 8192;
 #pragma unroll
-                for (int kk = 0; kk < 8; ++kk)
-                    mma_f16_ts(tmem + kColO, tmem + kColS + 64 * (jt & 1) + (kk < 4 ? 0 : 32) + 8 * (kk & 3),
-                               smem_desc(va + (kk & 3) * 2048, 8192, 1024, kLayoutSw128), idesc_pv,
+                for (int kk = 0; kk < 4; ++kk)
+                    mma_f16_ts(tmem + kColO, tmem + kColS + 64 * (jt & 1) + 8 * kk,
+                               smem_desc(va + kk * 2048, 8192, 1024, kLayoutSw128), idesc_pv,
                                (jt > 0 || kk > 0) ? 1u : 0u);
                 mma_commit(&kvempty[stage]);
                 mma_commit(&pvdone[jt & 1]);
@@ -364,7 +395,8 @@ mla_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const Params p) {
                 const uint32_t kv_par = (j / kStages) & 1;
                 const long long t0 = clock64();
                 while (qk || pv) {
-                    if (pv && mbar_test(&pfull[(j - 1) & 1], ((j - 1) >> 1) & 1)) {
+                    if (pv && mbar_test(&pfull[(j - 1) & 1], ((j - 1) >> 1) & 1) &&
+                        mbar_test(&vconv[(j - 1) & 1], ((j - 1) >> 1) & 1)) {
                         tc_fence_after();
                         issue_pv(j - 1);
                         pv = false;
@@ -465,16 +497,13 @@ mla_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const Params p) {
             const bool warp_rescale = __any_sync(0xffffffffu, need) && j > 0;
             const float msub = m_run == -INFINITY ? 0.f : m_run;   // exp2(-inf) = +0
             float ls[4] = {0.f, 0.f, 0.f, 0.f};
-            uint32_t ph[32], pl[32];
+            uint32_t pk[32];
 #pragma unroll
             for (int i = 0; i < 64; i += 2) {
                 const float e0 = fast_exp2(fmaf(x[i], sc, -msub));
                 const float e1 = fast_exp2(fmaf(x[i + 1], sc, -msub));
                 ls[(i >> 1) & 3] += e0 + e1;
-                const float v0 = kFp8 ? e0 * cs[i] : e0, v1 = kFp8 ? e1 * cs[i + 1] : e1;
-                const uint32_t hi = pack_bf16(v0, v1);
-                ph[i / 2] = hi;
-                pl[i / 2] = pack_bf16(v0 - __uint_as_float(hi << 16), v1 - __uint_as_float(hi & 0xFFFF0000u));
+                pk[i / 2] = kFp8 ? pack_f16(e0 * cs[i], e1 * cs[i + 1]) : pack_f16(e0, e1);
             }
             l_run = l_run * alpha + ((ls[0] + ls[1]) + (ls[2] + ls[3]));
             // ---- O may be rescaled only once the previous PV has finished
@@ -491,8 +520,7 @@ mla_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const Params p) {
                     tmem_st32(lane_base + kColO + cc * 32, o);
                 }
             }
-            tmem_st32(lane_base + sb_col, ph);
-            tmem_st32(lane_base + sb_col + 32, pl);
+            tmem_st32(lane_base + sb_col, pk);
             tmem_st_wait();
             tc_fence_before();
             mbar_arrive(&pfull[j & 1]);
