@@ -260,25 +260,24 @@ indexer_fp8_tc_kernel(const __grid_constant__ CUtensorMap tm_k,
                     tmem_ld32(tbase + qi * kHeads, v0);
                     tmem_ld32(tbase + qi * kHeads + 32, v1);
                     tmem_ld_wait();
+                    // sum_h w_h * ReLU(D_h) in 8 independent partial sums (a single
+                    // chain of 64 dependent FMAs would dominate the tile's time)
                     const float4* w4 = reinterpret_cast<const float4*>(w_run + qi * kHeads);
-                    float acc = 0.f;
+                    float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
 #pragma unroll
                     for (int h4 = 0; h4 < 8; ++h4) {
-                        const float4 wa = w4[h4];
-                        acc = fmaf(wa.x, fmaxf(__uint_as_float(v0[4 * h4 + 0]), 0.f), acc);
-                        acc = fmaf(wa.y, fmaxf(__uint_as_float(v0[4 * h4 + 1]), 0.f), acc);
-                        acc = fmaf(wa.z, fmaxf(__uint_as_float(v0[4 * h4 + 2]), 0.f), acc);
-                        acc = fmaf(wa.w, fmaxf(__uint_as_float(v0[4 * h4 + 3]), 0.f), acc);
+                        const float4 wa = w4[h4], wb = w4[8 + h4];
+                        const int e = (h4 & 1) * 4;
+                        acc[e + 0] = fmaf(wa.x, fmaxf(__uint_as_float(v0[4 * h4 + 0]), 0.f), acc[e + 0]);
+                        acc[e + 1] = fmaf(wa.y, fmaxf(__uint_as_float(v0[4 * h4 + 1]), 0.f), acc[e + 1]);
+                        acc[e + 2] = fmaf(wa.z, fmaxf(__uint_as_float(v0[4 * h4 + 2]), 0.f), acc[e + 2]);
+                        acc[e + 3] = fmaf(wa.w, fmaxf(__uint_as_float(v0[4 * h4 + 3]), 0.f), acc[e + 3]);
+                        acc[e + 0] = fmaf(wb.x, fmaxf(__uint_as_float(v1[4 * h4 + 0]), 0.f), acc[e + 0]);
+                        acc[e + 1] = fmaf(wb.y, fmaxf(__uint_as_float(v1[4 * h4 + 1]), 0.f), acc[e + 1]);
+                        acc[e + 2] = fmaf(wb.z, fmaxf(__uint_as_float(v1[4 * h4 + 2]), 0.f), acc[e + 2]);
+                        acc[e + 3] = fmaf(wb.w, fmaxf(__uint_as_float(v1[4 * h4 + 3]), 0.f), acc[e + 3]);
                     }
-#pragma unroll
-                    for (int h4 = 0; h4 < 8; ++h4) {
-                        const float4 wa = w4[8 + h4];
-                        acc = fmaf(wa.x, fmaxf(__uint_as_float(v1[4 * h4 + 0]), 0.f), acc);
-                        acc = fmaf(wa.y, fmaxf(__uint_as_float(v1[4 * h4 + 1]), 0.f), acc);
-                        acc = fmaf(wa.z, fmaxf(__uint_as_float(v1[4 * h4 + 2]), 0.f), acc);
-                        acc = fmaf(wa.w, fmaxf(__uint_as_float(v1[4 * h4 + 3]), 0.f), acc);
-                    }
-                    res[qi] = acc;
+                    res[qi] = ((acc[0] + acc[4]) + (acc[1] + acc[5])) + ((acc[2] + acc[6]) + (acc[3] + acc[7]));
                 }
                 tc_fence_before();
                 __syncwarp();

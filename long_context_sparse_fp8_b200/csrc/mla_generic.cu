@@ -104,31 +104,47 @@ mla_generic_kernel(const void* __restrict__ q, int heads, int d_qk, int d_v, flo
 
 // Merge of split partials: o = sum_i exp(lse_i - lse) o_i with lse = log sum_i exp(lse_i).
 // One thread per 4 output values of one (query, head); a block covers 2 heads x 512.
+// With NS > 0 (= nsplit, known at compile time) every partial a thread needs is
+// loaded before any is used, so the loads overlap instead of forming a dependent
+// chain; NS = 0 handles any nsplit <= 16 the same way in a fixed-size frame.
+template <int NS>
 __global__ void __launch_bounds__(256)
 mla_combine_kernel(const float* __restrict__ o_part, const float* __restrict__ lse_part,
-                   int nsplit, int heads, int d_v, void* __restrict__ out, int out_dtype,
+                   int nsplit_rt, int heads, int d_v, void* __restrict__ out, int out_dtype,
                    float* __restrict__ lse) {
+    constexpr int kMaxSplit = NS > 0 ? NS : 16;
+    const int nsplit = NS > 0 ? NS : nsplit_rt;
     const int t = blockIdx.x;
     const int per_head = d_v / 4;                       // threads per head
     const int h = blockIdx.y * (blockDim.x / per_head) + threadIdx.x / per_head;
     const int d4 = threadIdx.x % per_head;
     if (h >= heads) return;
+    float li[kMaxSplit];
+    float4 ov[kMaxSplit];
+#pragma unroll
+    for (int i = 0; i < kMaxSplit; ++i) {
+        if (i < nsplit) {
+            const long long pb = ((long long)t * nsplit + i) * heads + h;
+            li[i] = __ldg(lse_part + pb);
+            ov[i] = __ldg(reinterpret_cast<const float4*>(o_part + pb * d_v) + d4);
+        }
+    }
     float mx = -INFINITY;
-    for (int i = 0; i < nsplit; ++i)
-        mx = fmaxf(mx, __ldg(lse_part + ((long long)t * nsplit + i) * heads + h));
+#pragma unroll
+    for (int i = 0; i < kMaxSplit; ++i)
+        if (i < nsplit) mx = fmaxf(mx, li[i]);
     float wsum = 0.f;
     float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-    for (int i = 0; i < nsplit; ++i) {
-        const long long pb = ((long long)t * nsplit + i) * heads + h;
-        const float li = __ldg(lse_part + pb);
-        if (li == -INFINITY) continue;
-        const float wgt = __expf(li - mx);
-        wsum += wgt;
-        const float4 v = __ldg(reinterpret_cast<const float4*>(o_part + pb * d_v) + d4);
-        acc.x = fmaf(wgt, v.x, acc.x);
-        acc.y = fmaf(wgt, v.y, acc.y);
-        acc.z = fmaf(wgt, v.z, acc.z);
-        acc.w = fmaf(wgt, v.w, acc.w);
+#pragma unroll
+    for (int i = 0; i < kMaxSplit; ++i) {
+        if (i < nsplit && li[i] != -INFINITY) {
+            const float wgt = __expf(li[i] - mx);
+            wsum += wgt;
+            acc.x = fmaf(wgt, ov[i].x, acc.x);
+            acc.y = fmaf(wgt, ov[i].y, acc.y);
+            acc.z = fmaf(wgt, ov[i].z, acc.z);
+            acc.w = fmaf(wgt, ov[i].w, acc.w);
+        }
     }
     const float inv = wsum > 0.f ? 1.0f / wsum : 0.f;
     const long long ob = ((long long)t * heads + h) * d_v + 4 * d4;
@@ -165,8 +181,17 @@ cudaError_t launch_mla_combine(const float* o_part, const float* lse_part, int t
     const int per_head = d_v / 4;
     const int heads_per_block = per_head >= 256 ? 1 : 256 / per_head;
     dim3 grid(total_q, (heads + heads_per_block - 1) / heads_per_block);
-    mla_combine_kernel<<<grid, per_head * heads_per_block, 0, st>>>(o_part, lse_part, nsplit,
-                                                                   heads, d_v, out, out_dtype, lse);
+    const int threads = per_head * heads_per_block;
+#define DSA_COMBINE(N) mla_combine_kernel<N><<<grid, threads, 0, st>>>(o_part, lse_part, nsplit, \
+                                                                    heads, d_v, out, out_dtype, lse)
+    switch (nsplit) {
+        case 2: DSA_COMBINE(2); break;
+        case 3: DSA_COMBINE(3); break;
+        case 4: DSA_COMBINE(4); break;
+        case 8: DSA_COMBINE(8); break;
+        default: DSA_COMBINE(0); break;
+    }
+#undef DSA_COMBINE
     return cudaGetLastError();
 }
 
