@@ -12,9 +12,11 @@
 // accumulator.  Each epilogue thread owns one key (one TMEM lane) and reduces its
 // row: sum_h w[row,h] * max(D, 0), then applies the key's and the query's scale.
 //
-// Roles (192 threads): warp 0 issues TMA loads (pages through the block table into
-// a 4-stage ring of 128-byte-swizzled tiles), warp 1 allocates TMEM and issues the
-// MMAs (double-buffered accumulators), warps 2-5 drain TMEM and write the logits.
+// Roles: warp 0 issues TMA loads (pages through the block table into a 4-stage ring
+// of 128-byte-swizzled tiles), warp 1 allocates TMEM and issues the MMAs (double-
+// buffered accumulators), the epilogue warps drain TMEM and write the logits: one
+// warpgroup for one query row per CTA (2 CTAs per SM), two warpgroups for four rows
+// (1 CTA per SM: the accumulators fill TMEM; each warpgroup reduces two rows).
 //
 // Grid: x = groups of G consecutive query rows (G = 1 for decode-like batches,
 // 4 otherwise; a group that spans sequences is processed as per-sequence runs),
@@ -33,7 +35,12 @@ constexpr int kTileKeys = 128;
 constexpr int kStages = 4;
 constexpr int kTileBytes = kTileKeys * kDim;       // 16 KB
 constexpr int kRowBytes = kHeads * kDim;            // one query row: 8 KB
-constexpr int kThreads = 192;
+// 2 producer warps + EPI epilogue warpgroups: EPI = 1 for one query row per CTA
+// (64 accumulator columns, 2 CTAs per SM), EPI = 2 for four rows (the double-
+// buffered 2 x 256-column accumulator fills TMEM: 1 CTA per SM, and each warpgroup
+// reduces two of the four rows of every tile).
+template <int EPI>
+constexpr int threads_for() { return 64 + 128 * EPI; }
 
 struct Params {
     const float* w;
@@ -92,7 +99,8 @@ __device__ __forceinline__ int page_of(const Params& p, int b, int s, int* bad) 
     return page;
 }
 
-__global__ void __launch_bounds__(kThreads, 2)
+template <int EPI>
+__global__ void __launch_bounds__(threads_for<EPI>(), EPI == 1 ? 2 : 1)
 indexer_fp8_tc_kernel(const __grid_constant__ CUtensorMap tm_k,
                       const __grid_constant__ CUtensorMap tm_q, Params p) {
     extern __shared__ uint8_t smem_raw[];
@@ -124,7 +132,7 @@ indexer_fp8_tc_kernel(const __grid_constant__ CUtensorMap tm_k,
         }
         for (int i = 0; i < 2; ++i) {
             mbar_init(&tfull[i], 1);
-            mbar_init(&tempty[i], 4);   // one arrive per epilogue warp
+            mbar_init(&tempty[i], 4 * EPI);   // one arrive per epilogue warp
         }
         mbar_init(qfull, 1);
         mbar_init(qempty, 1);
@@ -141,7 +149,7 @@ indexer_fp8_tc_kernel(const __grid_constant__ CUtensorMap tm_k,
     {   // head weights of the CTA's rows, loaded once (no per-run barrier needed)
         const int t_begin = blockIdx.x * p.G;
         const int nrow = min(p.G, p.bv.total_q - t_begin);
-        for (int i = threadIdx.x; i < nrow * kHeads; i += kThreads)
+        for (int i = threadIdx.x; i < nrow * kHeads; i += threads_for<EPI>())
             w_s[i] = __ldg(p.w + (long long)t_begin * kHeads + i);
     }
     tc_fence_before();
@@ -229,6 +237,9 @@ indexer_fp8_tc_kernel(const __grid_constant__ CUtensorMap tm_k,
         // ------------------------------------------------------------ epilogue
         const int quarter = warp & 3;                 // TMEM lane quarter this warp may access
         const int row = quarter * 32 + lane;          // key row within the tile
+        const int q_lo = EPI == 2 ? 2 * ((warp - 2) >> 2) : 0;   // query rows of this warp
+        constexpr int kRows = EPI == 2 ? 2 : 4;
+        const int q_hi = q_lo + kRows;
         int it = 0;
         bool alive = true;
         Run run;
@@ -254,7 +265,8 @@ indexer_fp8_tc_kernel(const __grid_constant__ CUtensorMap tm_k,
                 float res[4] = {0.f, 0.f, 0.f, 0.f};
                 const uint32_t tbase = tmem_base + ((uint32_t)(quarter * 32) << 16) + buf * ncols_buf;
 #pragma unroll
-                for (int qi = 0; qi < 4; ++qi) {
+                for (int u = 0; u < kRows; ++u) {
+                    const int qi = q_lo + u;
                     if (qi >= run.r) break;
                     uint32_t v0[32], v1[32];
                     tmem_ld32(tbase + qi * kHeads, v0);
@@ -277,17 +289,18 @@ indexer_fp8_tc_kernel(const __grid_constant__ CUtensorMap tm_k,
                         acc[e + 2] = fmaf(wb.z, fmaxf(__uint_as_float(v1[4 * h4 + 2]), 0.f), acc[e + 2]);
                         acc[e + 3] = fmaf(wb.w, fmaxf(__uint_as_float(v1[4 * h4 + 3]), 0.f), acc[e + 3]);
                     }
-                    res[qi] = ((acc[0] + acc[4]) + (acc[1] + acc[5])) + ((acc[2] + acc[6]) + (acc[3] + acc[7]));
+                    res[u] = ((acc[0] + acc[4]) + (acc[1] + acc[5])) + ((acc[2] + acc[6]) + (acc[3] + acc[7]));
                 }
                 tc_fence_before();
                 __syncwarp();
                 if (lane == 0) mbar_arrive(&tempty[buf]);
 #pragma unroll
-                for (int qi = 0; qi < 4; ++qi) {
+                for (int u = 0; u < kRows; ++u) {
+                    const int qi = q_lo + u;
                     if (qi >= run.r) break;
                     const int pos = run.pos_lo + qi;
                     float* dst = p.logits + (long long)(run.t0 + qi) * p.ld + s;
-                    if (s <= pos) *dst = bad ? -INFINITY : res[qi] * ks * qs[qi];
+                    if (s <= pos) *dst = bad ? -INFINITY : res[u] * ks * qs[qi];
                     else if (s < p.ld) *dst = -INFINITY;
                 }
             }
@@ -335,11 +348,18 @@ cudaError_t launch_indexer_fp8_tc(const void* q, const float* q_scale, const flo
     Params p{w, q_scale, k.scale, k.table, k.num_pages, k.bt_stride, bv, logits, ld, G, C, check};
     const size_t smem = 1024 + kStages * kTileBytes + (size_t)G * kRowBytes +
                         (size_t)G * kHeads * sizeof(float) + 16 * sizeof(uint64_t) + 16;
-    e = cudaFuncSetAttribute(indexer_fp8_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             (int)smem);
-    if (e != cudaSuccess) return e;
     dim3 grid(groups, chunks);
-    indexer_fp8_tc_kernel<<<grid, kThreads, smem, st>>>(tm_k, tm_q, p);
+    if (G == 1) {
+        e = cudaFuncSetAttribute(indexer_fp8_tc_kernel<1>,
+                                 cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+        if (e != cudaSuccess) return e;
+        indexer_fp8_tc_kernel<1><<<grid, threads_for<1>(), smem, st>>>(tm_k, tm_q, p);
+    } else {
+        e = cudaFuncSetAttribute(indexer_fp8_tc_kernel<2>,
+                                 cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+        if (e != cudaSuccess) return e;
+        indexer_fp8_tc_kernel<2><<<grid, threads_for<2>(), smem, st>>>(tm_k, tm_q, p);
+    }
     return cudaGetLastError();
 }
 
