@@ -15,13 +15,14 @@
 //      histogram fixes the bin b1 of the k-th key: every key in a higher bin is in.
 //   2. One sweep over 32-key groups writes a selection bitmap straight from warp
 //      ballots (bit set = bin above b1) and appends the keys of bin b1 with their
-//      positions to a candidate list C.
+//      positions to the sweeping warp's own segment of a candidate list C.
 //   3. Two radix passes (11 + 10 bits) over C fix the exact k-th key T and how many
 //      keys equal to T are needed; keys above T get their bit, and the equal keys
 //      go to a second bitmap from which the lowest positions are taken.
 //   4. A block scan over the bitmap's popcounts turns it into the ascending list.
-// If C would overflow (thousands of keys in one bin, e.g. equal scores), step 2 is
-// replaced by radix passes over the whole row and one marking sweep.  Rows longer
+// If C would overflow (thousands of keys in one bin, e.g. equal scores, or more than
+// a segment's worth in one warp's share), steps 2-3 fall back to radix passes over
+// the whole row and one marking sweep.  Rows longer
 // than the bitmap capacity use a second kernel that refines over the whole row and
 // emits in two ordered sweeps.
 #include "kernels.h"
@@ -34,7 +35,8 @@ constexpr int kWarps = kThreads / 32;
 constexpr int kTopBits = 11;
 constexpr uint32_t kLowMask = (1u << (32 - kTopBits)) - 1u;   // 21 low key bits
 constexpr int kCopies = 4;                 // interleaved copies of the first histogram
-constexpr int kCandCap = 4096;             // candidates: low 21 key bits + position
+constexpr int kCandCap = 8192;             // candidates: low 21 key bits + position
+constexpr int kSeg = kCandCap / 32;        // per-warp candidate segment
 constexpr int kMaxWords = 8192;            // bitmap words: rows up to 262144 keys
 constexpr int kSmemLimit = 232448;
 constexpr int kStaticReserve = 1024;
@@ -48,7 +50,8 @@ __device__ __forceinline__ uint32_t order_key(float f) {
 
 struct Shared {
     int warp_sums[kWarps + 1];
-    int bin, above, count, n_c;
+    int bin, above, count;
+    int seg_n[32];            // candidates found by each warp
 };
 
 // Block-wide exclusive prefix sum of one int per thread; *total gets the sum.
@@ -130,17 +133,18 @@ struct Row {
 // One radix refinement pass over n keys: histogram (copy 0) of bits
 // [shift, shift+nbits) of the keys matching prefix/pmask, then the bin of the
 // remaining-th largest; *count = keys in that bin.
-template <class KeyF>
-__device__ __forceinline__ void refine(Shared& sh, int* hist, int n, KeyF key_of, int shift,
+// for_each(f) calls f(key) for this thread's share of the keys.
+template <class ForEach>
+__device__ __forceinline__ void refine(Shared& sh, int* hist, ForEach for_each, int shift,
                                        int nbits, uint32_t& prefix, uint32_t& pmask,
                                        int& remaining, int* count) {
     const int nb = 1 << nbits, tid = threadIdx.x;
     for (int i = tid; i < nb; i += kThreads) hist[i] = 0;
     __syncthreads();
-    for (int i = tid; i < n; i += kThreads) {
-        const uint32_t key = key_of(i);
-        if ((key & pmask) == prefix) atomicAdd(&hist[(key >> shift) & (nb - 1)], 1);
-    }
+    const uint32_t pf = prefix, pm = pmask;
+    for_each([&](uint32_t key) {
+        if ((key & pm) == pf) atomicAdd(&hist[(key >> shift) & (nb - 1)], 1);
+    });
     __syncthreads();
     int above;
     const int bin = find_bin(sh, hist, 1, nb, remaining, &above, count);
@@ -232,7 +236,6 @@ topk_kernel(const float* __restrict__ logits, long long ld, BatchView bv, int k,
 
     // ---- 1. stage + top-bit histogram ------------------------------------------
     for (int i = tid; i < kCopies * 2048; i += kThreads) hist[i] = 0;
-    if (tid == 0) sh.n_c = 0;
     __syncthreads();
     stage_and_histogram(grow, n, skeys, stage_cap, hist);
     __syncthreads();
@@ -242,8 +245,15 @@ topk_kernel(const float* __restrict__ logits, long long ld, BatchView bv, int k,
     uint32_t T;                         // the k-th largest key
     int n_eq;                           // keys equal to T
 
-    if (n_cand <= kCandCap) {
-        // ---- 2. bitmap of the higher bins; candidates of bin b1 -> C -------------
+    // whole-row iteration for the radix passes of the fallback
+    auto row_each = [&](auto f) {
+        for (int i = tid; i < n; i += kThreads) f(row(i));
+    };
+    bool fast = n_cand <= kCandCap;
+    if (fast) {
+        // ---- 2. bitmap of the higher bins; candidates of bin b1 -> per-warp segments
+        // of C (no shared counter: one would serialise every warp on one address)
+        int c_at = 0;
         for (int g0 = warp; g0 < words; g0 += 4 * kWarps) {
             uint32_t kk[4];
 #pragma unroll
@@ -265,27 +275,31 @@ topk_kernel(const float* __restrict__ logits, long long ld, BatchView bv, int k,
                     eqmap[g] = 0u;
                 }
                 if (mc) {
-                    int base = 0;
-                    if (lane == 0) base = atomicAdd(&sh.n_c, __popc(mc));
-                    base = __shfl_sync(0xffffffffu, base, 0);
-                    if (cand) {
-                        const int c = base + __popc(mc & ((1u << lane) - 1u));
-                        ckey[c] = kk[u] & kLowMask;
-                        cpos[c] = i;
+                    const int c = c_at + __popc(mc & ((1u << lane) - 1u));
+                    if (cand && c < kSeg) {
+                        ckey[warp * kSeg + c] = kk[u] & kLowMask;
+                        cpos[warp * kSeg + c] = i;
                     }
+                    c_at += __popc(mc);
                 }
             }
         }
-        __syncthreads();
+        if (lane == 0) sh.seg_n[warp] = c_at;
+        fast = !__syncthreads_or(c_at > kSeg);   // a full segment: take the fallback
+    }
+    if (fast) {
         // ---- 3. exact threshold among the candidates; mark them ------------------
+        const int seg_cnt = sh.seg_n[warp];        // <= kSeg here
+        auto cand_each = [&](auto f) {
+            for (int c = lane; c < seg_cnt; c += 32) f(ckey[warp * kSeg + c]);
+        };
         uint32_t prefix = 0u, pmask = 0u;
-        auto cand_key = [&](int i) { return ckey[i]; };
-        refine(sh, hist, n_cand, cand_key, 10, 11, prefix, pmask, remaining, &n_eq);
-        refine(sh, hist, n_cand, cand_key, 0, 10, prefix, pmask, remaining, &n_eq);
+        refine(sh, hist, cand_each, 10, 11, prefix, pmask, remaining, &n_eq);
+        refine(sh, hist, cand_each, 0, 10, prefix, pmask, remaining, &n_eq);
         T = prefix;
-        for (int c = tid; c < n_cand; c += kThreads) {
-            const uint32_t key = ckey[c];
-            const int p = cpos[c];
+        for (int c = lane; c < seg_cnt; c += 32) {
+            const uint32_t key = ckey[warp * kSeg + c];
+            const int p = cpos[warp * kSeg + c];
             if (key > T) atomicOr(&bitmap[p >> 5], 1u << (p & 31));
             else if (key == T) atomicOr(&eqmap[p >> 5], 1u << (p & 31));
         }
@@ -293,8 +307,8 @@ topk_kernel(const float* __restrict__ logits, long long ld, BatchView bv, int k,
         // ---- fallback: refine over the whole row, then one marking sweep ---------
         uint32_t prefix = b1 << (32 - kTopBits);
         uint32_t pmask = ~kLowMask;
-        refine(sh, hist, n, row, 10, 11, prefix, pmask, remaining, &n_eq);
-        refine(sh, hist, n, row, 0, 10, prefix, pmask, remaining, &n_eq);
+        refine(sh, hist, row_each, 10, 11, prefix, pmask, remaining, &n_eq);
+        refine(sh, hist, row_each, 0, 10, prefix, pmask, remaining, &n_eq);
         T = prefix;
         for (int g0 = warp; g0 < words; g0 += 4 * kWarps) {
             uint32_t kk[4];
@@ -380,8 +394,11 @@ topk_long_kernel(const float* __restrict__ logits, long long ld, BatchView bv, i
     const uint32_t b1 = (uint32_t)find_bin(sh, hist, kCopies, 2048, k, &n_def, &cnt);
     int remaining = k - n_def;
     uint32_t prefix = b1 << (32 - kTopBits), pmask = ~kLowMask;
-    refine(sh, hist, n, row, 10, 11, prefix, pmask, remaining, &cnt);
-    refine(sh, hist, n, row, 0, 10, prefix, pmask, remaining, &cnt);
+    auto row_each = [&](auto f) {
+        for (int i = tid; i < n; i += kThreads) f(row(i));
+    };
+    refine(sh, hist, row_each, 10, 11, prefix, pmask, remaining, &cnt);
+    refine(sh, hist, row_each, 0, 10, prefix, pmask, remaining, &cnt);
     const uint32_t T = prefix;
     const int need_eq = remaining;
 
