@@ -197,10 +197,12 @@ dsa_status_t mla_check(const void* q, dsa_dtype_t q_dtype, int heads, int d_qk, 
 cudaError_t mla_launch(const MlaPlan& plan, const void* q, int heads, int d_qk, int d_v,
                        float scale, const BatchView& bv, const int* idx, int k, int nsplit,
                        void* out, int out_dtype, float* lse, float* o_part, float* lse_part,
-                       int* check, cudaStream_t st) {
+                       int* check, cudaStream_t st, bool pdl = false) {
+    // (pdl: the tensor-core kernel waits for its predecessor before reading idx; the
+    // CUDA-core kernel does not, so it is always launched plainly)
     if (plan.kind == MlaKind::kTensorCore)
         return launch_mla_tc(q, scale, plan.kv, bv, idx, k, nsplit, out, lse, o_part, lse_part,
-                             check, st);
+                             check, st, pdl);
     return launch_mla_generic(q, heads, d_qk, d_v, scale, plan.kv, bv, idx, k, nsplit, out,
                               out_dtype, lse, o_part, lse_part, check, st);
 }
@@ -239,18 +241,19 @@ dsa_status_t mla_decode_validate(const BatchView& bv, int heads, int d_v, int k,
 cudaError_t mla_decode_launch(const MlaPlan& plan, const void* q, int heads, int d_qk, int d_v,
                               float scale, const BatchView& bv, const int* idx, int k, void* out,
                               dsa_dtype_t out_dtype, float* lse, void* ws, int* check,
-                              cudaStream_t st) {
+                              cudaStream_t st, bool pdl = false) {
     const int ns = decode_splits(bv.total_q, k);
     if (ns == 1)
         return mla_launch(plan, q, heads, d_qk, d_v, scale, bv, idx, k, 1, out, out_dtype, lse,
-                          nullptr, nullptr, check, st);
+                          nullptr, nullptr, check, st, pdl);
     float* o_part = static_cast<float*>(ws);
     float* l_part = reinterpret_cast<float*>(
         static_cast<char*>(ws) + align_up((size_t)bv.total_q * ns * heads * d_v * 4, 256));
     cudaError_t e = mla_launch(plan, q, heads, d_qk, d_v, scale, bv, idx, k, ns, nullptr,
-                               out_dtype, nullptr, o_part, l_part, check, st);
+                               out_dtype, nullptr, o_part, l_part, check, st, pdl);
     if (e != cudaSuccess) return e;
-    return launch_mla_combine(o_part, l_part, bv.total_q, ns, heads, d_v, out, out_dtype, lse, st);
+    return launch_mla_combine(o_part, l_part, bv.total_q, ns, heads, d_v, out, out_dtype, lse, st,
+                              pdl);
 }
 
 long long decode_ld(int max_seq_len) { return ((long long)max_seq_len + 63) / 64 * 64; }
@@ -431,10 +434,13 @@ DSA_API dsa_status_t dsa_decode(const void* q_idx, dsa_dtype_t q_idx_dtype,
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     if (e == cudaSuccess)
         e = indexer_launch(q_idx, q_idx_scale, w, idx_heads, idx_dim, kc, bv, logits, ld, check, st);
-    if (e == cudaSuccess) e = launch_topk(logits, ld, bv, k, sel, check, st);
+    // top-k, attention and merge start as programmatic dependents of the kernel before
+    // them (each waits for its predecessor's results; the indexer, launched plainly,
+    // orders the whole chain after the caller's earlier work on the stream)
+    if (e == cudaSuccess) e = launch_topk(logits, ld, bv, k, sel, check, st, true);
     if (e == cudaSuccess)
         e = mla_decode_launch(plan, q, heads, d_qk, d_v, softmax_scale, bv, sel, k, out, out_dtype,
-                              lse, mla_ws, check, st);
+                              lse, mla_ws, check, st, true);
     return e == cudaSuccess ? ok() : cuda_fail(e, "decode launch");
 }
 

@@ -34,6 +34,14 @@ struct CacheView {
     int dtype;
 };
 
+// Programmatic dependent launch.  A kernel launched with programmatic stream
+// serialization may start while its predecessor in the stream still runs: it must
+// execute pdl_wait() before touching anything the predecessor writes (returns at
+// once when there is no such predecessor).  pdl_trigger() lets the successor be
+// scheduled before this grid ends.
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void pdl_trigger() { asm volatile("griddepcontrol.launch_dependents;" :::); }
+
 __device__ __forceinline__ void report(int* check, int code) {
     if (check) atomicCAS(check, 0, code);
 }

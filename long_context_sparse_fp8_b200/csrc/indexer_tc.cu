@@ -89,16 +89,6 @@ __device__ __forceinline__ bool get_run(const Params& p, int k, Run* out, bool s
     return false;
 }
 
-__device__ __forceinline__ int page_of(const Params& p, int b, int s, int* bad) {
-    const int page = __ldg(p.table + (long long)b * p.bt_stride + s / 64);
-    if (page < 0 || (long long)page >= p.num_pages) {
-        *bad = 1;
-        return 0;
-    }
-    *bad = 0;
-    return page;
-}
-
 template <int EPI>
 __global__ void __launch_bounds__(threads_for<EPI>(), EPI == 1 ? 2 : 1)
 indexer_fp8_tc_kernel(const __grid_constant__ CUtensorMap tm_k,
@@ -174,19 +164,46 @@ indexer_fp8_tc_kernel(const __grid_constant__ CUtensorMap tm_k,
                 mbar_arrive_expect_tx(qfull, p.G * kRowBytes);
                 tma_load_2d(q_tile, &tm_q, 0, run.t0 * kHeads, qfull);
                 const int pos_hi = run.pos_lo + run.r - 1;
-                for (int j = run.j0; j < run.j1; ++j, ++it) {
-                    const int stage = it % kStages;
-                    const uint32_t ph = (it / kStages) & 1;
-                    if (!mbar_wait(&empty[stage], ph ^ 1, p.check)) { alive = false; break; }
-                    int bad0, bad1 = 0;
-                    const int p0 = page_of(p, run.b, j * kTileKeys, &bad0);
-                    const bool two = j * kTileKeys + 64 <= pos_hi;
-                    const int p1 = two ? page_of(p, run.b, j * kTileKeys + 64, &bad1) : 0;
-                    if (bad0 | bad1) report(p.check, kCheckBadPage);
-                    mbar_arrive_expect_tx(&full[stage], two ? kTileBytes : kTileBytes / 2);
-                    uint8_t* dst = a_tiles + stage * kTileBytes;
-                    tma_load_2d(dst, &tm_k, 0, p0 * 64, &full[stage]);
-                    if (two) tma_load_2d(dst + kTileBytes / 2, &tm_k, 0, p1 * 64, &full[stage]);
+                // block-table entries of the run's tiles, loaded four tiles at a time and
+                // one group ahead of their use (a lookup right before each TMA would put a
+                // global-load latency on every tile)
+                const int* trow = p.table + (long long)run.b * p.bt_stride;
+                auto load_pages = [&](int jt, int (&pg)[8]) {
+#pragma unroll
+                    for (int u = 0; u < 4; ++u) {
+                        const int s0 = (jt + u) * kTileKeys;
+                        const bool in = jt + u < run.j1;
+                        pg[2 * u] = in ? __ldg(trow + s0 / 64) : 0;
+                        pg[2 * u + 1] = (in && s0 + 64 <= pos_hi) ? __ldg(trow + s0 / 64 + 1) : 0;
+                    }
+                };
+                int cur[8], nxt[8];
+                load_pages(run.j0, cur);
+                load_pages(run.j0 + 4, nxt);
+                for (int j4 = run.j0; alive && j4 < run.j1; j4 += 4) {
+#pragma unroll
+                    for (int u = 0; u < 4; ++u) {
+                        const int j = j4 + u;
+                        if (j >= run.j1) break;
+                        const int stage = it % kStages;
+                        const uint32_t ph = (it / kStages) & 1;
+                        if (!mbar_wait(&empty[stage], ph ^ 1, p.check)) { alive = false; break; }
+                        const bool two = j * kTileKeys + 64 <= pos_hi;
+                        int p0 = cur[2 * u], p1 = cur[2 * u + 1];
+                        const bool bad0 = p0 < 0 || (long long)p0 >= p.num_pages;
+                        const bool bad1 = two && (p1 < 0 || (long long)p1 >= p.num_pages);
+                        if (bad0 | bad1) report(p.check, kCheckBadPage);
+                        if (bad0) p0 = 0;
+                        if (bad1) p1 = 0;
+                        mbar_arrive_expect_tx(&full[stage], two ? kTileBytes : kTileBytes / 2);
+                        uint8_t* dst = a_tiles + stage * kTileBytes;
+                        tma_load_2d(dst, &tm_k, 0, p0 * 64, &full[stage]);
+                        if (two) tma_load_2d(dst + kTileBytes / 2, &tm_k, 0, p1 * 64, &full[stage]);
+                        ++it;
+                    }
+#pragma unroll
+                    for (int i = 0; i < 8; ++i) cur[i] = nxt[i];
+                    load_pages(j4 + 8, nxt);
                 }
             }
             // drain: every issued stage has been consumed (its empty phase completed)
@@ -239,7 +256,6 @@ indexer_fp8_tc_kernel(const __grid_constant__ CUtensorMap tm_k,
         const int row = quarter * 32 + lane;          // key row within the tile
         const int q_lo = EPI == 2 ? 2 * ((warp - 2) >> 2) : 0;   // query rows of this warp
         constexpr int kRows = EPI == 2 ? 2 : 4;
-        const int q_hi = q_lo + kRows;
         int it = 0;
         bool alive = true;
         Run run;
@@ -251,15 +267,29 @@ indexer_fp8_tc_kernel(const __grid_constant__ CUtensorMap tm_k,
             for (int i = 0; i < 4; ++i)
                 qs[i] = (i < run.r && p.q_scale) ? __ldg(p.q_scale + run.t0 + i) : 1.0f;
             const int pos_hi = run.pos_lo + run.r - 1;
+            // this key's block-table entry two tiles ahead and its scale one tile ahead
+            // (a table -> scale load chain per tile would stall every tile)
+            const int* trow = p.table + (long long)run.b * p.bt_stride;
+            auto tbl = [&](int jt) -> int {
+                const int sk = jt * kTileKeys + row;
+                return (jt < run.j1 && sk <= pos_hi) ? __ldg(trow + sk / 64) : 0;
+            };
+            auto scl = [&](int jt, int pg) -> float {
+                const int sk = jt * kTileKeys + row;
+                if (jt >= run.j1 || sk > pos_hi || pg < 0 || (long long)pg >= p.num_pages) return 0.f;
+                return p.k_scale ? __ldg(p.k_scale + (long long)pg * 64 + (sk & 63)) : 1.0f;
+            };
+            int pg1 = tbl(run.j0), pg2 = tbl(run.j0 + 1);
+            float ks1 = scl(run.j0, pg1);
             for (int j = run.j0; j < run.j1; ++j, ++it) {
                 const int buf = it & 1;
                 const int s = j * kTileKeys + row;
-                float ks = 0.f;
-                int bad = 1;
-                if (s <= pos_hi) {
-                    const int page = page_of(p, run.b, s, &bad);
-                    ks = p.k_scale ? __ldg(p.k_scale + (long long)page * 64 + (s & 63)) : 1.0f;
-                }
+                const int page = pg1;
+                const float ks = ks1;
+                const int bad = (s <= pos_hi && (page < 0 || (long long)page >= p.num_pages)) ? 1 : 0;
+                pg1 = pg2;
+                pg2 = tbl(j + 2);
+                ks1 = scl(j + 1, pg1);
                 if (!mbar_wait_warp(&tfull[buf], (it >> 1) & 1, p.check)) { alive = false; break; }
                 tc_fence_after();
                 float res[4] = {0.f, 0.f, 0.f, 0.f};

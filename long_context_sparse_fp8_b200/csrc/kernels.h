@@ -2,12 +2,32 @@
 // in include/dsa.h validates arguments and then calls these.
 #pragma once
 
+#include <utility>
+
 #include <cuda.h>
 #include <cuda_runtime.h>
 
 #include "common.cuh"
 
 namespace dsa {
+
+// Launch; with pdl, as a programmatic dependent of the previous kernel in the stream
+// (the kernel must then pdl_wait() before reading that kernel's results).
+template <typename... KArgs, typename... Args>
+cudaError_t launch_kernel(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem,
+                          cudaStream_t st, bool pdl, Args&&... args) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = grid;
+    cfg.blockDim = block;
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = pdl ? 1 : 0;
+    return cudaLaunchKernelEx(&cfg, kern, std::forward<Args>(args)...);
+}
 
 constexpr int kIndexerPage = 64;
 constexpr int kNumSMs = 148;
@@ -30,7 +50,7 @@ cudaError_t launch_indexer_fp8_tc(const void* q, const float* q_scale, const flo
 
 // Per-row top-k by radix select.
 cudaError_t launch_topk(const float* logits, long long ld, const BatchView& bv, int k, int* idx,
-                        int* check, cudaStream_t st);
+                        int* check, cudaStream_t st, bool pdl = false);
 
 // Sparse MLA on CUDA cores (fp32 q/KV).  nsplit > 1 writes partials (o/l, lse) to
 // o_part [T][nsplit][heads][d_v] / lse_part [T][nsplit][heads] instead of out/lse.
@@ -42,7 +62,7 @@ cudaError_t launch_mla_generic(const void* q, int heads, int d_qk, int d_v, floa
 // Sparse MLA on tcgen05 tensor cores: bf16 q, bf16 or fp8 KV, 128 heads, 576 / 512.
 cudaError_t launch_mla_tc(const void* q, float scale, const CacheView& kv, const BatchView& bv,
                           const int* idx, int k, int nsplit, void* out, float* lse, float* o_part,
-                          float* lse_part, int* check, cudaStream_t st);
+                          float* lse_part, int* check, cudaStream_t st, bool pdl = false);
 
 // Size of the fixed device array behind dsa_sparse_mla_decode_noalloc
 // (equals DSA_NOALLOC_SCRATCH_BYTES in include/dsa.h).
@@ -54,6 +74,6 @@ cudaError_t static_scratch(void** ptr);
 // Log-sum-exp merge of split partials into out (out_dtype) and lse.
 cudaError_t launch_mla_combine(const float* o_part, const float* lse_part, int total_q, int nsplit,
                                int heads, int d_v, void* out, int out_dtype, float* lse,
-                               cudaStream_t st);
+                               cudaStream_t st, bool pdl = false);
 
 }  // namespace dsa

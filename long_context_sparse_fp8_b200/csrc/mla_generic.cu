@@ -118,6 +118,7 @@ mla_combine_kernel(const float* __restrict__ o_part, const float* __restrict__ l
     const int per_head = d_v / 4;                       // threads per head
     const int h = blockIdx.y * (blockDim.x / per_head) + threadIdx.x / per_head;
     const int d4 = threadIdx.x % per_head;
+    pdl_wait();                                         // partials of the previous kernel
     if (h >= heads) return;
     float li[kMaxSplit];
     float4 ov[kMaxSplit];
@@ -176,22 +177,18 @@ cudaError_t launch_mla_generic(const void* q, int heads, int d_qk, int d_v, floa
 
 cudaError_t launch_mla_combine(const float* o_part, const float* lse_part, int total_q, int nsplit,
                                int heads, int d_v, void* out, int out_dtype, float* lse,
-                               cudaStream_t st) {
+                               cudaStream_t st, bool pdl) {
     // d_v % 4 == 0 and d_v <= 512 (validated by the callers)
     const int per_head = d_v / 4;
     const int heads_per_block = per_head >= 256 ? 1 : 256 / per_head;
     dim3 grid(total_q, (heads + heads_per_block - 1) / heads_per_block);
     const int threads = per_head * heads_per_block;
-#define DSA_COMBINE(N) mla_combine_kernel<N><<<grid, threads, 0, st>>>(o_part, lse_part, nsplit, \
-                                                                    heads, d_v, out, out_dtype, lse)
-    switch (nsplit) {
-        case 2: DSA_COMBINE(2); break;
-        case 3: DSA_COMBINE(3); break;
-        case 4: DSA_COMBINE(4); break;
-        case 8: DSA_COMBINE(8); break;
-        default: DSA_COMBINE(0); break;
-    }
-#undef DSA_COMBINE
+    auto kern = nsplit == 2 ? mla_combine_kernel<2> : nsplit == 3 ? mla_combine_kernel<3>
+              : nsplit == 4 ? mla_combine_kernel<4> : nsplit == 8 ? mla_combine_kernel<8>
+                                                                  : mla_combine_kernel<0>;
+    cudaError_t e = launch_kernel(kern, grid, dim3(threads), 0, st, pdl, o_part, lse_part, nsplit,
+                                  heads, d_v, out, out_dtype, lse);
+    if (e != cudaSuccess) return e;
     return cudaGetLastError();
 }
 

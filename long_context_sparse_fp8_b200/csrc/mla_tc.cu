@@ -189,6 +189,7 @@ mla_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const Params p) {
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + kNumBars);
 
     const int warp = threadIdx.x >> 5;
+    pdl_trigger();
     const int vh = blockIdx.x & 1;                   // which half of the V columns
     const int cid = blockIdx.x >> 1;
     const int t = cid / p.nsplit, split = cid % p.nsplit;
@@ -269,6 +270,7 @@ mla_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const Params p) {
         // pipeline over the group's own tiles: slots of tiles j and j+2, the table
         // entry of tile j+4 and the index of tile j+6 are in flight at tile j
         int sl_cur = -1, sl_next = -1, raw_n2 = kSkip, idx_n3 = -1;
+        pdl_wait();                                  // the selection may come from the previous kernel
         if (grp < n_tiles) {
             const int x0 = fetch_idx(grp), x1 = fetch_idx(grp + 2), x2 = fetch_idx(grp + 4);
             idx_n3 = fetch_idx(grp + 6);
@@ -584,7 +586,7 @@ mla_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const Params p) {
 
 cudaError_t launch_mla_tc(const void* q, float scale, const CacheView& kv, const BatchView& bv,
                           const int* idx, int k, int nsplit, void* out, float* lse, float* o_part,
-                          float* lse_part, int* check, cudaStream_t st) {
+                          float* lse_part, int* check, cudaStream_t st, bool pdl) {
     Params p;
     p.q = reinterpret_cast<const uint4*>(q);
     p.kv = reinterpret_cast<const uint8_t*>(kv.data);
@@ -614,7 +616,8 @@ cudaError_t launch_mla_tc(const void* q, float scale, const CacheView& kv, const
                                          (int)kSmemBytes);
     if (e != cudaSuccess) return e;
     dim3 grid(2 * bv.total_q * nsplit);
-    kern<<<grid, kThreads, kSmemBytes, st>>>(tm_q, p);
+    e = launch_kernel(kern, grid, dim3(kThreads), kSmemBytes, st, pdl, tm_q, p);
+    if (e != cudaSuccess) return e;
     return cudaGetLastError();
 }
 

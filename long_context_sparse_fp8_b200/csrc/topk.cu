@@ -219,6 +219,7 @@ topk_kernel(const float* __restrict__ logits, long long ld, BatchView bv, int k,
     __shared__ Shared sh;
 
     const int t = blockIdx.x, tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    pdl_trigger();
     int* out = idx + (long long)t * k;
     const RowInfo ri = row_info(bv, t, check);
     if (!ri.ok) {
@@ -233,6 +234,7 @@ topk_kernel(const float* __restrict__ logits, long long ld, BatchView bv, int k,
     const float* grow = logits + (long long)t * ld;
     const Row row{grow, skeys, stage_cap};
     const int words = (n + 31) >> 5;
+    pdl_wait();                                  // the logits may come from the previous kernel
 
     // ---- 1. stage + top-bit histogram ------------------------------------------
     for (int i = tid; i < kCopies * 2048; i += kThreads) hist[i] = 0;
@@ -386,6 +388,7 @@ topk_long_kernel(const float* __restrict__ logits, long long ld, BatchView bv, i
     }
     const float* grow = logits + (long long)t * ld;
     const Row row{grow, skeys, stage_cap};
+    pdl_wait();
     for (int i = tid; i < kCopies * 2048; i += kThreads) hist[i] = 0;
     __syncthreads();
     stage_and_histogram(grow, n, skeys, stage_cap, hist);
@@ -441,7 +444,7 @@ topk_long_kernel(const float* __restrict__ logits, long long ld, BatchView bv, i
 }  // namespace
 
 cudaError_t launch_topk(const float* logits, long long ld, const BatchView& bv, int k, int* idx,
-                        int* check, cudaStream_t st) {
+                        int* check, cudaStream_t st, bool pdl) {
     const int hist_bytes = kCopies * 2048 * 4;
     const int words = ((bv.max_seq_len + 31) / 32 + 3) & ~3;
     if (words <= kMaxWords) {
@@ -452,15 +455,18 @@ cudaError_t launch_topk(const float* logits, long long ld, const BatchView& bv, 
         cudaError_t e = cudaFuncSetAttribute(topk_kernel,
                                              cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
         if (e != cudaSuccess) return e;
-        topk_kernel<<<bv.total_q, kThreads, smem, st>>>(logits, ld, bv, k, idx, check, words,
-                                                        stage);
+        e = launch_kernel(topk_kernel, dim3(bv.total_q), dim3(kThreads), smem, st, pdl, logits, ld,
+                          bv, k, idx, check, words, stage);
+        if (e != cudaSuccess) return e;
     } else {
         const int stage = (kSmemLimit - kStaticReserve - hist_bytes) / 4 & ~3;
         const size_t smem = (size_t)hist_bytes + (size_t)stage * 4;
         cudaError_t e = cudaFuncSetAttribute(topk_long_kernel,
                                              cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
         if (e != cudaSuccess) return e;
-        topk_long_kernel<<<bv.total_q, kThreads, smem, st>>>(logits, ld, bv, k, idx, check, stage);
+        e = launch_kernel(topk_long_kernel, dim3(bv.total_q), dim3(kThreads), smem, st, pdl, logits,
+                          ld, bv, k, idx, check, stage);
+        if (e != cudaSuccess) return e;
     }
     return cudaGetLastError();
 }
