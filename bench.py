@@ -33,6 +33,7 @@ ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
 
 import long_context_sparse_fp8_b200 as L  # noqa: E402
+from long_context_sparse_fp8_b200 import replicas as R  # noqa: E402
 from long_context_sparse_fp8_b200 import workloads as W  # noqa: E402
 
 METRIC = "DSA tokens/s (decode & prefill) on 1 B200; % of HBM / tensor-core roofline"
@@ -58,33 +59,6 @@ def parse():
 
 
 # ----------------------------------------------------------------------------- plumbing
-def dist_setup(args):
-    world = int(os.environ.get("WORLD_SIZE", "1"))
-    rank = int(os.environ.get("RANK", "0"))
-    local = int(os.environ.get("LOCAL_RANK", "0"))
-    if world > 1:
-        import datetime
-        torch.cuda.set_device(local)
-        torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
-    else:
-        torch.cuda.set_device(0)
-    return rank, world
-
-
-def barrier(world):
-    if world > 1:
-        torch.distributed.barrier()
-    torch.cuda.synchronize()
-
-
-def max_over_ranks(x: float, world: int) -> float:
-    if world == 1:
-        return x
-    t = torch.tensor([x], device="cuda", dtype=torch.float64)
-    torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-    return float(t.item())
-
-
 class ClockSampler:
     """SM clock and clock-event reasons of this process's GPU, read through NVML every
     millisecond or so by a background thread while the timed loop runs (the loop lasts
@@ -299,11 +273,10 @@ def timed_loop(fn_list, steps, flush, stream):
     return [[e[j].elapsed_time(e[j + 1]) for j in range(len(fn_list))] for e in evs]
 
 
-def run_dsa(args, rank, world):
+def run_dsa(args, rank, world, dev):
     spec_fn, mode = WORKLOADS[args.workload]
     spec = spec_fn()
-    spec.seed += 1000 * rank  # independent replica inputs per rank
-    dev = torch.device("cuda", torch.cuda.current_device())
+    spec.seed = R.replica_seed(spec.seed, rank)  # independent replica inputs per rank
     wl = W.make(spec, device=dev)
     st = Step(wl, mode)
     stream = torch.cuda.current_stream()
@@ -316,19 +289,19 @@ def run_dsa(args, rank, world):
         raise RuntimeError("device check recorded an error during warm-up")
 
     # ---- headline: K fused steps
-    barrier(world)
+    R.barrier(world, dev)
     with ClockSampler(torch.cuda.current_device()) as clk:
         step_ms = [sum(x) for x in timed_loop([st.fused], args.steps, flush, stream)]
-    barrier(world)
+    R.barrier(world, dev)
     ms = statistics.mean(step_ms)
-    ms_max = max_over_ranks(ms, world)
+    ms_max = R.max_over_ranks(ms, world, dev)
     tokens = spec.total_q
-    value = tokens * world / (ms_max / 1e3)
+    value = R.job_throughput(tokens, ms_max, world)
 
     # ---- per-stage breakdown of the same kernels (roofline)
-    barrier(world)
+    R.barrier(world, dev)
     stage_ms = timed_loop(st.stages(), args.steps, flush, stream)
-    barrier(world)
+    R.barrier(world, dev)
     names = ["indexer", "topk", "mla"]
     mean_stage = {n: statistics.mean(r[j] for r in stage_ms) for j, n in enumerate(names)}
     work = st.work()
@@ -366,11 +339,11 @@ def run_dsa(args, rank, world):
 
         for _ in range(3):
             e2e_step()
-        barrier(world)
+        R.barrier(world, dev)
         e_ms = statistics.mean(sum(x) for x in timed_loop([e2e_step], args.steps, flush, stream))
-        e_ms = max_over_ranks(e_ms, world)
+        e_ms = R.max_over_ranks(e_ms, world, dev)
         h2d = sum(t.numel() * t.element_size() for t in (h_qidx, h_w, h_q))
-        e2e = {"value": round(tokens * world / (e_ms / 1e3), 1), "unit": "tokens/s",
+        e2e = {"value": round(R.job_throughput(tokens, e_ms, world), 1), "unit": "tokens/s",
                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": h_out.numel() * 2,
                "ms_per_step": round(e_ms, 4)}
 
@@ -484,14 +457,13 @@ def main():
         if res is not None:
             print(json.dumps(res), flush=True)
         return
-    rank, world = dist_setup(args)
+    rank, world, dev = R.setup()
     try:
-        res = run_dsa(args, rank, world)
+        res = run_dsa(args, rank, world, dev)
         if rank == 0:
             print(json.dumps(res), flush=True)
     finally:
-        if world > 1:
-            torch.distributed.destroy_process_group()
+        R.teardown(world)
 
 
 if __name__ == "__main__":
