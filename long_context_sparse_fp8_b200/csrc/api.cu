@@ -132,9 +132,9 @@ dsa_status_t indexer_validate(const void* q, dsa_dtype_t q_dtype, const float* q
 
 cudaError_t indexer_launch(const void* q, const float* q_scale, const float* w, int heads, int dim,
                            const CacheView& kc, const BatchView& bv, float* logits, long long ld,
-                           int* check, cudaStream_t st) {
+                           int* check, cudaStream_t st, bool pdl = false) {
     if (kc.dtype == kE4M3)  // validated: 64 heads x 128 dims
-        return launch_indexer_fp8_tc(q, q_scale, w, kc, bv, logits, ld, check, st);
+        return launch_indexer_fp8_tc(q, q_scale, w, kc, bv, logits, ld, check, st, pdl);
     return launch_indexer_generic(q, q_scale, w, heads, dim, kc, bv, logits, ld, check, st);
 }
 
@@ -433,10 +433,14 @@ DSA_API dsa_status_t dsa_decode(const void* q_idx, dsa_dtype_t q_idx_dtype,
     cudaError_t e = check_word(&check);
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     if (e == cudaSuccess)
-        e = indexer_launch(q_idx, q_idx_scale, w, idx_heads, idx_dim, kc, bv, logits, ld, check, st);
-    // top-k, attention and merge start as programmatic dependents of the kernel before
-    // them (each waits for its predecessor's results; the indexer, launched plainly,
-    // orders the whole chain after the caller's earlier work on the stream)
+        e = indexer_launch(q_idx, q_idx_scale, w, idx_heads, idx_dim, kc, bv, logits, ld, check, st,
+                           true);
+    // every kernel of the chain starts as a programmatic dependent of the kernel before
+    // it and waits for that kernel before touching memory it may write: the tensor-core
+    // indexer before reading anything (its predecessor is the caller's earlier work),
+    // top-k before the logits, attention before the selection, the merge before the
+    // partials; each kernel finishes only after its own wait, so the chain is ordered
+    // after everything earlier on the stream (the CUDA-core indexer ignores pdl)
     if (e == cudaSuccess) e = launch_topk(logits, ld, bv, k, sel, check, st, true);
     if (e == cudaSuccess)
         e = mla_decode_launch(plan, q, heads, d_qk, d_v, softmax_scale, bv, sel, k, out, out_dtype,

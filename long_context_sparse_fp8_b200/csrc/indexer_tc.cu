@@ -110,6 +110,7 @@ indexer_fp8_tc_kernel(const __grid_constant__ CUtensorMap tm_k,
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(qempty + 1);
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    pdl_trigger();
     const int ncols_buf = p.G * kHeads;                     // accumulator columns per buffer
     const uint32_t tmem_cols = ncols_buf * 2 <= 128 ? 128u : (ncols_buf * 2 <= 256 ? 256u : 512u);
 
@@ -136,6 +137,7 @@ indexer_fp8_tc_kernel(const __grid_constant__ CUtensorMap tm_k,
         prefetch_tmap(&tm_k);
         prefetch_tmap(&tm_q);
     }
+    pdl_wait();   // launched as a dependent: every input may come from the previous kernel
     {   // head weights of the CTA's rows, loaded once (no per-run barrier needed)
         const int t_begin = blockIdx.x * p.G;
         const int nrow = min(p.G, p.bv.total_q - t_begin);
@@ -353,7 +355,7 @@ cudaError_t make_map(CUtensorMap* m, const void* base, unsigned long long rows, 
 
 cudaError_t launch_indexer_fp8_tc(const void* q, const float* q_scale, const float* w,
                                   const CacheView& k, const BatchView& bv, float* logits,
-                                  long long ld, int* check, cudaStream_t st) {
+                                  long long ld, int* check, cudaStream_t st, bool pdl) {
     const int T = bv.total_q;
     const int G = T <= 2 * bv.num_seqs ? 1 : 4;
     const int groups = (T + G - 1) / G;
@@ -383,12 +385,16 @@ cudaError_t launch_indexer_fp8_tc(const void* q, const float* q_scale, const flo
         e = cudaFuncSetAttribute(indexer_fp8_tc_kernel<1>,
                                  cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
         if (e != cudaSuccess) return e;
-        indexer_fp8_tc_kernel<1><<<grid, threads_for<1>(), smem, st>>>(tm_k, tm_q, p);
+        e = launch_kernel(indexer_fp8_tc_kernel<1>, grid, dim3(threads_for<1>()), smem, st, pdl,
+                          tm_k, tm_q, p);
+        if (e != cudaSuccess) return e;
     } else {
         e = cudaFuncSetAttribute(indexer_fp8_tc_kernel<2>,
                                  cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
         if (e != cudaSuccess) return e;
-        indexer_fp8_tc_kernel<2><<<grid, threads_for<2>(), smem, st>>>(tm_k, tm_q, p);
+        e = launch_kernel(indexer_fp8_tc_kernel<2>, grid, dim3(threads_for<2>()), smem, st, pdl,
+                          tm_k, tm_q, p);
+        if (e != cudaSuccess) return e;
     }
     return cudaGetLastError();
 }

@@ -46,7 +46,7 @@ cudaError_t launch_indexer_generic(const void* q, const float* q_scale, const fl
 // Lightning Indexer on tcgen05 tensor cores (fp8 e4m3 q/k, 64 heads x 128 dims).
 cudaError_t launch_indexer_fp8_tc(const void* q, const float* q_scale, const float* w,
                                   const CacheView& k, const BatchView& bv, float* logits,
-                                  long long ld, int* check, cudaStream_t st);
+                                  long long ld, int* check, cudaStream_t st, bool pdl = false);
 
 // Per-row top-k by radix select.
 cudaError_t launch_topk(const float* logits, long long ld, const BatchView& bv, int k, int* idx,
