@@ -145,6 +145,28 @@ def test_topk_ties_and_long_rows(n, k, kind):
         assert np.array_equal(np.sort(got[0]), np.arange(k))
 
 
+def test_topk_candidates_concentrated_in_one_warp():
+    # The keys of the k-th key's top-bit bin all sit in 32-key groups that one warp of
+    # the top-k CTA sweeps (every 32nd group), so that warp's candidate segment
+    # overflows and the row must take the whole-row fallback -- same result required.
+    n, k = 60000, 2048
+    pos = np.arange(n)
+    row = np.zeros(n, dtype=np.float32)
+    mine = np.flatnonzero((pos // 32) % 32 == 0)[:900]         # 900 candidates, one warp
+    row[mine] = 5.0 + (np.arange(len(mine)) % 97) * 1e-3        # same 11-bit bin, many ties
+    top = np.setdiff1d(pos, mine)[::37][:1500]                  # 1500 keys above that bin
+    row[top] = 10.0
+    ld = (n + 3) // 4 * 4
+    logits = torch.full((1, ld), float("nan"), device="cuda")
+    logits[0, :n] = torch.from_numpy(row).cuda()
+    batch = L.Batch(torch.tensor([0, 1], dtype=torch.int32, device="cuda"),
+                    torch.tensor([n], dtype=torch.int32, device="cuda"), 1, n)
+    idx = torch.empty(1, k, dtype=torch.int32, device="cuda")
+    L.dsa_topk(logits, batch, k, idx)
+    got = idx.cpu().numpy()
+    H.check_topk(got, logits.cpu().numpy(), logits.cpu().numpy(), np.array([n - 1]), k)
+
+
 def test_device_check_reports_bad_index_and_page():
     spec = W.Spec(name="chk", seq_lens=[300], nq=[4], topk=64, seed=5)
     wl = W.make(spec, device="cuda")
