@@ -118,7 +118,8 @@ def test_small_k_and_fp32_mla_split():
                                       (70000, 2048, "normal"), (2048, 2048, "normal"),
                                       (100000, 4096, "equal"), (50000, 2048, "coarse"),
                                       (20000, 2048, "normal"), (9000, 100, "coarse"),
-                                      (300000, 2048, "normal"), (300000, 2048, "three")])
+                                      (300000, 2048, "normal"), (300000, 2048, "three"),
+                                      (100000, 65536, "normal"), (65536, 65536, "coarse")])
 def test_topk_ties_and_long_rows(n, k, kind):
     g = torch.Generator(device="cuda").manual_seed(n + k)
     if kind == "equal":
