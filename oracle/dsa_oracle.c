@@ -274,3 +274,100 @@ int oracle_sparse_mla(const void* q, int q_dtype, int heads, int d_qk, int d_v,
 }
 
 int oracle_num_threads(void) { return omp_get_max_threads(); }
+
+/* ------------------------------------------------------------ cache writes
+ * The caches the indexer and the attention read are filled token by token:
+ * "SGLang Day-0 support for DeepSeek-V3.2" (winzheng.jp review), section
+ * "DeepSeek Sparse Attention" -- the indexer keeps a key & key_scale cache
+ * (page size 64) and the sparse operator a token-level cache (page size 1);
+ * its "Future work" section and its launch line's KV_CACHE_STORE_FP8 switch:
+ * the KV cache may be stored in FP8, halving the bytes attention reads;
+ * "DeepSeek-V3.2-Exp DSA deployment guide" (m.nxbn.cn), section 3.1:
+ * fp8_e4m3 KV cache.  The problem fixes the FP8 scaling: one fp32 scale per
+ * token, amax / 448 (448 = the largest finite e4m3 magnitude).
+ */
+
+/* fp32 -> OCP e4m3, round to nearest (ties to even), magnitudes that round
+ * above 448 saturate to 448, the sign is kept (also on zero), NaN -> 0x7F.
+ * Written from the bit layout: normal codes are (1 + m/8) * 2^(E-7) for
+ * E = 1..15 (E = 15, m = 7 is NaN), subnormal codes m * 2^-9. */
+uint8_t oracle_f32_to_e4m3(float f) {
+    if (isnan(f)) return 0x7F;
+    uint8_t sign = signbit(f) ? 0x80 : 0x00;
+    double a = fabs((double)f);
+    if (a >= 448.0) return sign | 0x7E;
+    if (a == 0.0) return sign;
+    int e2;
+    frexp(a, &e2);          /* a = fr * 2^e2, fr in [0.5, 1): floor(log2 a) = e2 - 1 */
+    int ex = e2 - 1;
+    if (ex < -6) ex = -6;   /* below 2^-6 the spacing stays 2^-9 (subnormals) */
+    double quantum = ldexp(1.0, ex - 3);
+    double n = nearbyint(a / quantum);   /* a / quantum is exact; default mode = ties to even */
+    double v = n * quantum;
+    if (v > 448.0) v = 448.0;
+    if (v == 0.0) return sign;
+    if (v < ldexp(1.0, -6))
+        return sign | (uint8_t)(v / ldexp(1.0, -9));              /* subnormal: m in 1..7 */
+    frexp(v, &e2);
+    ex = e2 - 1;                                                   /* -6 .. 8 */
+    int m = (int)(v / ldexp(1.0, ex - 3)) - 8;                     /* 0 .. 7 */
+    return sign | (uint8_t)(((ex + 7) << 3) | m);
+}
+
+/* fp32 -> bf16 bits, round to nearest even (NaN keeps a quiet NaN). */
+uint16_t oracle_f32_to_bf16(float f) {
+    uint32_t u;
+    memcpy(&u, &f, sizeof u);
+    if (isnan(f)) return (uint16_t)((u >> 16) | 0x40);
+    uint32_t lower = u & 0xFFFF, upper = u >> 16;
+    if (lower > 0x8000 || (lower == 0x8000 && (upper & 1))) upper += 1;
+    return (uint16_t)upper;
+}
+
+/*
+ * Writes n tokens into a cache seen as num_rows rows of dim elements.
+ *   x             [n][dim] of x_dtype (fp32 or bf16)
+ *   slot_mapping  [n]: cache row of token i (page * page_size + row in page);
+ *                 a negative entry skips the token
+ *   cache_data    [num_rows][dim] of cache_dtype; cache_scale [num_rows] fp32
+ * FP8 cache: amax = max_e |x_e| (fp32), scale = amax / 448 in fp32 (1 when
+ * amax = 0), code_e = e4m3(x_e / scale) with the quotient an IEEE fp32
+ * division.  BF16 cache: x rounded to bf16.  FP32 cache: x as is.  The scale
+ * of a non-FP8 cache is left untouched.  Returns -1 (after writing the valid
+ * tokens) if a slot is >= num_rows.
+ */
+int oracle_cache_store(const void* x, int x_dtype, int64_t n, int dim,
+                       const int64_t* slot_mapping, void* cache_data, int cache_dtype,
+                       float* cache_scale, int64_t num_rows) {
+    int bad = 0;
+    for (int64_t i = 0; i < n; ++i) {
+        int64_t slot = slot_mapping[i];
+        if (slot < 0) continue;
+        if (slot >= num_rows) {
+            bad = 1;
+            continue;
+        }
+        float* row = (float*)malloc((size_t)dim * sizeof(float));
+        for (int d = 0; d < dim; ++d) row[d] = (float)load_elem(x, x_dtype, i * dim + d);
+        if (cache_dtype == OR_E4M3) {
+            float amax = 0.0f;
+            for (int d = 0; d < dim; ++d)
+                if (fabsf(row[d]) > amax) amax = fabsf(row[d]);
+            volatile float scale = amax > 0.0f ? amax / 448.0f : 1.0f;
+            uint8_t* dst = (uint8_t*)cache_data + slot * dim;
+            for (int d = 0; d < dim; ++d) {
+                volatile float quotient = row[d] / scale;
+                dst[d] = oracle_f32_to_e4m3(quotient);
+            }
+            cache_scale[slot] = scale;
+        } else if (cache_dtype == OR_BF16) {
+            uint16_t* dst = (uint16_t*)cache_data + slot * dim;
+            for (int d = 0; d < dim; ++d) dst[d] = oracle_f32_to_bf16(row[d]);
+        } else {
+            float* dst = (float*)cache_data + slot * dim;
+            for (int d = 0; d < dim; ++d) dst[d] = row[d];
+        }
+        free(row);
+    }
+    return bad ? -1 : 0;
+}

@@ -13,6 +13,9 @@ Sources of each definition (page title and section):
     "DeepSeek-V3.2-Exp DSA deployment guide" (m.nxbn.cn) sections 1, 3.1, 5.1.
   * bf16 q with a bf16 or fp8 KV cache: "DeepSeek V3.2 usage guide" (SGLang
     docs), attention-kernel section.
+  * cache writes (the page-64 key & key_scale cache, the token-level KV cache,
+    FP8 storage): "SGLang Day-0 support for DeepSeek-V3.2", sections "DeepSeek
+    Sparse Attention" and "Future work"; deployment guide section 3.1.
 
 Dtype codes: 0 = fp32, 1 = bf16 (raw uint16 bits), 2 = fp8 e4m3 (raw bytes).
 Parity pins for every function live in tests/test_oracle_pins.py; none of the
@@ -69,6 +72,12 @@ def _load():
                                               i32, P, P, P, i32, P, i64, P, P]
             lib.oracle_sparse_mla.restype = i32
             lib.oracle_num_threads.restype = i32
+            lib.oracle_f32_to_e4m3.argtypes = [ctypes.c_float]
+            lib.oracle_f32_to_e4m3.restype = ctypes.c_uint8
+            lib.oracle_f32_to_bf16.argtypes = [ctypes.c_float]
+            lib.oracle_f32_to_bf16.restype = ctypes.c_uint16
+            lib.oracle_cache_store.argtypes = [P, i32, i64, i32, P, P, i32, P, i64]
+            lib.oracle_cache_store.restype = i32
             _lib = lib
     return _lib
 
@@ -172,3 +181,33 @@ def decode(idx_args: dict, k: int, mla_args: dict, cu_q, seq_lens, ld, rows=None
     sel = topk(logits, cu_q, seq_lens, k, rows=rows)
     out, lse = sparse_mla(cu_q=cu_q, seq_lens=seq_lens, idx=sel, rows=rows, **mla_args)
     return logits, sel, out, lse
+
+
+def f32_to_e4m3(x: float) -> int:
+    """One fp32 value to its e4m3 code (RNE, saturating at 448, sign kept)."""
+    return int(_load().oracle_f32_to_e4m3(float(x)))
+
+
+def f32_to_bf16(x: float) -> int:
+    """One fp32 value to bf16 bits (RNE)."""
+    return int(_load().oracle_f32_to_bf16(float(x)))
+
+
+def cache_store(x, x_dtype, slot_mapping, cache_data, cache_dtype, cache_scale):
+    """Writes the rows of ``x`` [n, dim] into copies of ``cache_data`` [num_rows, dim]
+    (raw numpy of the cache dtype) and ``cache_scale`` [num_rows] (or None); returns
+    (data, scale).  Row i goes to cache row ``slot_mapping[i]``; negative skips."""
+    lib = _load()
+    x = _c(x)
+    n, dim = x.shape
+    slots = _c(slot_mapping, np.int64)
+    assert slots.shape == (n,)
+    data = np.array(cache_data, copy=True, order="C")
+    scale = None if cache_scale is None else np.array(cache_scale, dtype=np.float32, copy=True)
+    if cache_dtype == E4M3 and scale is None:
+        raise ValueError("an fp8 cache needs its scale array")
+    rc = lib.oracle_cache_store(_ptr(x), x_dtype, n, dim, _ptr(slots), _ptr(data), cache_dtype,
+                                _ptr(scale), data.shape[0])
+    if rc != 0:
+        raise ValueError("oracle_cache_store: slot outside [0, num_rows)")
+    return data, scale

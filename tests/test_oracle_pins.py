@@ -347,3 +347,142 @@ def test_mla_rejects_noncausal_index():
     kv = np.zeros((4, 4), np.float32)
     with pytest.raises(ValueError):
         _mla(q, kv, np.array([[3]], np.int32), [0, 1], [3], 1.0, 2)
+
+
+# ---------------------------------------------------------------- cache writes
+def _e4m3_values():
+    """Every finite e4m3 value (non-negative codes 0..0x7E), as float64."""
+    return np.array([O.e4m3_to_double(c) for c in range(0x7F)])
+
+
+def test_e4m3_encoder_matches_torch_cast():
+    """The oracle's encoder (bit layout + ties-to-even) against torch's float8 cast on
+    the codes themselves, every midpoint between neighbours (ties), one fp32 ulp on
+    either side of each midpoint, and random values across the whole range."""
+    v = _e4m3_values()
+    mids = (v[:-1] + v[1:]) / 2
+    m32 = mids.astype(np.float32)
+    xs = [v.astype(np.float32), m32, np.nextafter(m32, np.float32(np.inf)),
+          np.nextafter(m32, np.float32(0))]
+    g = np.random.default_rng(7)
+    mag = np.exp(g.uniform(np.log(1e-5), np.log(448.0), 20000)).astype(np.float32)
+    xs.append(mag)
+    x = np.concatenate(xs)
+    x = np.concatenate([x, -x, np.float32([0.0, -0.0, 448.0, -448.0])])
+    ours = np.array([O.f32_to_e4m3(float(a)) for a in x], dtype=np.uint8)
+    ref = _bits(torch.from_numpy(x).to(torch.float8_e4m3fn))
+    bad = np.nonzero(ours != ref)[0]
+    assert bad.size == 0, [(float(x[i]), hex(ours[i]), hex(ref[i])) for i in bad[:5]]
+
+
+def test_e4m3_encoder_round_trip_saturation_and_ties():
+    for c in range(256):
+        if c & 0x7F == 0x7F:
+            continue                                  # NaN codes
+        assert O.f32_to_e4m3(O.e4m3_to_double(c)) == c
+    assert O.f32_to_e4m3(448.0001) == 0x7E and O.f32_to_e4m3(-1e30) == 0xFE
+    assert O.f32_to_e4m3(float("inf")) == 0x7E       # saturating, not NaN
+    assert O.f32_to_e4m3(float("nan")) & 0x7F == 0x7F
+    assert O.f32_to_e4m3(2.0 ** -10) == 0x00          # tie 0 | 2^-9 -> even (0)
+    assert O.f32_to_e4m3(3 * 2.0 ** -10) == 0x02      # tie 2^-9 | 2^-8 -> even (2)
+    assert O.f32_to_e4m3(1.0625) == 0x38              # tie 1 | 1.125 -> 1
+    assert O.f32_to_e4m3(-1.1875) == 0x80 | 0x3A      # tie 1.125 | 1.25 -> 1.25
+    assert O.f32_to_e4m3(-1e-6) == 0x80               # underflow keeps the sign
+
+
+def test_bf16_encoder_matches_torch():
+    g = np.random.default_rng(8)
+    x = g.standard_normal(50000).astype(np.float32) * np.float32(3.0)
+    u = x.view(np.uint32)
+    ties = ((u & 0xFFFF0000) | 0x8000).view(np.float32)     # exact halfway cases
+    x = np.concatenate([x, ties, np.float32([0.0, -0.0, 1e-40, -3e38])])
+    ours = np.array([O.f32_to_bf16(float(a)) for a in x], dtype=np.uint16)
+    ref = _bits(torch.from_numpy(x).to(torch.bfloat16))
+    assert np.array_equal(ours, ref)
+
+
+def _cache(num_rows, dim, dtype):
+    g = np.random.default_rng(9)
+    raw = {O.E4M3: np.uint8, O.BF16: np.uint16, O.F32: np.float32}[dtype]
+    data = g.integers(0, 0x7E, (num_rows, dim)).astype(raw) if dtype != O.F32 else \
+        g.standard_normal((num_rows, dim)).astype(np.float32)
+    return data, g.uniform(0.5, 2.0, num_rows).astype(np.float32)
+
+
+def test_cache_store_fp8_scale_codes_and_untouched_rows():
+    """scale = amax / 448; the amax element becomes +-448 exactly; every code
+    decodes to x / scale within half a code step (1/16 relative, 2^-10 absolute in
+    the subnormal range); an all-zero row gets scale 1 and zero codes; rows the
+    slot mapping skips or does not name keep their bytes."""
+    g = np.random.default_rng(10)
+    n, dim, rows = 40, 576, 100
+    x = g.standard_normal((n, dim)).astype(np.float32)
+    x[3] *= 4.0
+    x[5] = 0.0
+    x[7] *= 1e-3
+    slots = g.permutation(rows)[:n].astype(np.int64)
+    slots[11] = -1
+    data0, scale0 = _cache(rows, dim, O.E4M3)
+    data, scale = O.cache_store(x, O.F32, slots, data0, O.E4M3, scale0)
+    for i in range(n):
+        s = slots[i]
+        if s < 0:
+            continue
+        amax = np.float32(np.abs(x[i]).max())
+        want = np.float32(amax / np.float32(448.0)) if amax > 0 else np.float32(1.0)
+        assert scale[s] == want
+        q = x[i] / want
+        dec = np.array([O.e4m3_to_double(c) for c in data[s]])
+        err = np.abs(dec - q)
+        assert np.all(err <= np.maximum(np.abs(q) / 16, 2.0 ** -10) + 1e-12), i
+        if amax > 0:
+            j = int(np.abs(x[i]).argmax())
+            assert data[s, j] == (0xFE if x[i, j] < 0 else 0x7E)
+        else:
+            assert np.all(data[s] == 0)
+    touched = set(int(s) for s in slots if s >= 0)
+    for r in range(rows):
+        if r not in touched:
+            assert np.array_equal(data[r], data0[r]) and scale[r] == scale0[r]
+
+
+def test_cache_store_bf16_and_f32_caches():
+    g = np.random.default_rng(11)
+    x = g.standard_normal((9, 128)).astype(np.float32)
+    slots = np.array([4, 0, -1, 8, 2, 7, -5, 1, 3], dtype=np.int64)
+    d0, s0 = _cache(10, 128, O.BF16)
+    d, s = O.cache_store(x, O.F32, slots, d0, O.BF16, s0)
+    ref = _bits(torch.from_numpy(x).to(torch.bfloat16))
+    for i, sl in enumerate(slots):
+        if sl >= 0:
+            assert np.array_equal(d[sl], ref[i])
+    assert np.array_equal(d[[5, 6, 9]], d0[[5, 6, 9]]) and np.array_equal(s, s0)
+    xb = ref                                          # bf16 input bits into a bf16 cache
+    d2, _ = O.cache_store(xb, O.BF16, slots, d0, O.BF16, None)
+    for i, sl in enumerate(slots):
+        if sl >= 0:
+            assert np.array_equal(d2[sl], xb[i])
+    f0, _ = _cache(10, 128, O.F32)
+    f, _ = O.cache_store(xb, O.BF16, slots, f0, O.F32, None)
+    wide = torch.from_numpy(xb.view(np.int16)).view(torch.bfloat16).float().numpy()
+    for i, sl in enumerate(slots):
+        if sl >= 0:
+            assert np.array_equal(f[sl], wide[i])
+
+
+def test_cache_store_bf16_input_same_codes_as_its_fp32_value():
+    """A bf16 row and the same values in fp32 quantise identically (the input is
+    widened exactly before amax and the quotients)."""
+    g = np.random.default_rng(12)
+    xf = torch.from_numpy(g.standard_normal((6, 128)).astype(np.float32)).to(torch.bfloat16)
+    slots = np.arange(6, dtype=np.int64)
+    d0, s0 = _cache(6, 128, O.E4M3)
+    a, sa = O.cache_store(_bits(xf), O.BF16, slots, d0, O.E4M3, s0)
+    b, sb = O.cache_store(xf.float().numpy(), O.F32, slots, d0, O.E4M3, s0)
+    assert np.array_equal(a, b) and np.array_equal(sa, sb)
+
+
+def test_cache_store_rejects_slot_past_the_end():
+    d0, s0 = _cache(4, 16, O.E4M3)
+    with pytest.raises(ValueError):
+        O.cache_store(np.ones((2, 16), np.float32), O.F32, np.array([1, 4]), d0, O.E4M3, s0)
