@@ -14,6 +14,10 @@ for the roofline.  Multi-GPU runs are independent replicas (one batch per rank, 
 data-path collective): value = all ranks' tokens / the slowest rank's time.
 
 `--impl reference` times the CPU oracle on a bounded sample of the same workload.
+
+`--workload store_L131072_fp8` times the cache writes instead: one step writes a
+131072-token prompt's indexer keys (page 64) and latent-KV rows (page 1) into FP8
+caches (dsa_cache_store, twice).
 """
 from __future__ import annotations
 
@@ -43,6 +47,7 @@ WORKLOADS = {
     "decode_b32_ctx8192": (W.decode_b32_8k, "decode"),
     "prefill_L32768_q8192": (W.prefill_32k, "prefill"),
     "decode_b64_ctx64k-128k_fp8kv": (W.decode_b64_128k, "decode"),
+    "store_L131072_fp8": (W.store_prompt_128k, "store"),
 }
 
 
@@ -275,6 +280,8 @@ def timed_loop(fn_list, steps, flush, stream):
 
 def run_dsa(args, rank, world, dev):
     spec_fn, mode = WORKLOADS[args.workload]
+    if mode == "store":
+        return run_store(args, rank, world, dev)
     spec = spec_fn()
     spec.seed = R.replica_seed(spec.seed, rank)  # independent replica inputs per rank
     wl = W.make(spec, device=dev)
@@ -433,6 +440,133 @@ def run_dsa(args, rank, world, dev):
     }
 
 
+# ----------------------------------------------------------------------------- cache writes
+def _store_bytes(x, out_elem):
+    """Algorithmic bytes of one store call: rows in, codes + scale out, the slot map."""
+    n, dim = x.shape
+    return n * (dim * x.element_size() + dim * out_elem + (4 if out_elem == 1 else 0) + 8)
+
+
+def run_store(args, rank, world, dev):
+    spec = W.store_prompt_128k()
+    spec.seed = R.replica_seed(spec.seed, rank)
+    wl = W.make_store(spec, device=dev)
+    stream = torch.cuda.current_stream()
+    flush = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    calls = [lambda: L.dsa_cache_store(wl.k_new, wl.k_slots, wl.k_pages, wl.k_scale),
+             lambda: L.dsa_cache_store(wl.kv_new, wl.kv_slots, wl.kv, wl.kv_scale)]
+
+    def step():
+        for c in calls:
+            c()
+
+    for _ in range(max(3, args.warmup)):
+        step()
+    torch.cuda.synchronize()
+    if L.dsa_device_check() != 0:
+        raise RuntimeError("device check recorded an error during warm-up")
+    R.barrier(world, dev)
+    with ClockSampler(torch.cuda.current_device()) as clk:
+        step_ms = [sum(x) for x in timed_loop([step], args.steps, flush, stream)]
+    R.barrier(world, dev)
+    ms_max = R.max_over_ranks(statistics.mean(step_ms), world, dev)
+    n = spec.n_tokens
+    value = R.job_throughput(n, ms_max, world)
+    stage_ms = timed_loop(calls, args.steps, flush, stream)
+    mean_stage = {nm: statistics.mean(r[j] for r in stage_ms)
+                  for j, nm in enumerate(["key_store", "kv_store"])}
+    kv_elem = wl.kv.element_size()
+    work = {"key_store": _store_bytes(wl.k_new, 1), "kv_store": _store_bytes(wl.kv_new, kv_elem)}
+    hbm_gbs, _, peak_kind = measured_peaks()
+    dom = "kv_store"
+    achieved = work[dom] / (mean_stage[dom] / 1e3) / 1e9
+    roof = {"bound": "hbm", "achieved": round(achieved, 1), "peak": hbm_gbs, "unit": "GB/s",
+            "frac": round(achieved / hbm_gbs, 4),
+            "traffic": ncu_traffic(args.workload, "cache_store.cu"), "kernel": dom,
+            "peak_source": f"{peak_kind} (burst)",
+            "stage_ms": {k: round(v, 4) for k, v in mean_stage.items()},
+            "algorithmic_bytes_per_launch": work[dom]}
+
+    # end to end: the rows and slot maps come from pinned host memory each step and
+    # the written per-token scales go back (neighbouring steps overlap on copy streams)
+    names = ("k_new", "kv_new", "k_slots", "kv_slots")
+    host = {k: getattr(wl, k).cpu().pin_memory() for k in names}
+    back = {"k_scale": torch.empty(wl.k_scale.shape).pin_memory(),
+            "kv_scale": torch.empty(wl.kv_scale.shape).pin_memory()}
+    h2d_s, d2h_s = torch.cuda.Stream(dev), torch.cuda.Stream(dev)
+    R.barrier(world, dev)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    done, ready = torch.cuda.Event(), torch.cuda.Event()
+    h2d_s.wait_stream(stream)
+    d2h_s.wait_stream(stream)
+    e0.record(stream)
+    for i in range(args.steps):
+        with torch.cuda.stream(h2d_s):
+            if i:
+                h2d_s.wait_event(done)
+            for k in names:
+                getattr(wl, k).copy_(host[k], non_blocking=True)
+            ready.record(h2d_s)
+        stream.wait_event(ready)
+        step()
+        done.record(stream)
+        with torch.cuda.stream(d2h_s):
+            d2h_s.wait_event(done)
+            back["k_scale"].copy_(wl.k_scale, non_blocking=True)
+            back["kv_scale"].copy_(wl.kv_scale, non_blocking=True)
+    stream.wait_stream(d2h_s)
+    e1.record(stream)
+    torch.cuda.synchronize(dev)
+    e_ms = R.max_over_ranks(e0.elapsed_time(e1) / args.steps, world, dev)
+    e2e = {"value": round(R.job_throughput(n, e_ms, world), 1), "unit": "tokens/s",
+           "h2d_bytes_per_step": sum(host[k].numel() * host[k].element_size() for k in names),
+           "d2h_bytes_per_step": sum(b.numel() * 4 for b in back.values()),
+           "ms_per_step": round(e_ms, 4),
+           "method": "pinned H2D of the new rows and slot maps, D2H of the written scales, "
+                     "every step; eager launches"}
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        cpu = _store_oracle(wl, args.cpu_seconds)
+    if L.dsa_device_check() != 0:
+        raise RuntimeError("device check recorded an error in the timed region")
+    return {
+        "metric": "cache-write tokens/s (indexer key + latent KV into FP8 caches) on 1 B200",
+        "value": round(value, 1), "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": round(ms_max, 5), "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "bf16 in, fp8 e4m3 + fp32 scale out",
+        "data": "synthetic (seeded N(0,1) rows, 1% x4)",
+        "config": {"workload": spec.name, "mode": "store", "tokens": n,
+                   "key": f"{spec.idx_dim} dims -> page-64 fp8 cache",
+                   "kv": f"{spec.d_qk} dims -> page-1 fp8 cache",
+                   "l2": "flushed between steps (256 MiB write)",
+                   "parallelism": f"replicas x{world}"},
+        "roofline": roof, "cpu_baseline": cpu, "e2e": e2e, "clocks": clk.summary(),
+        "gpu_launches": 2 * args.steps, "gpu_launches_note": "two cache_store launches per step",
+    }
+
+
+def _store_oracle(wl, seconds, rows=None):
+    """The oracle's cache write on a bounded token sample (both caches)."""
+    import numpy as np
+    from oracle import oracle as O
+    n = wl.spec.n_tokens
+    if rows is None:
+        rows = 4096
+    sel = np.arange(min(rows, n))
+    kd = wl.k_pages.view(torch.uint8).reshape(-1, wl.spec.idx_dim).cpu().numpy()
+    vd = wl.kv.view(torch.uint8).cpu().numpy()
+    ks, vs = wl.k_scale.reshape(-1).cpu().numpy(), wl.kv_scale.cpu().numpy()
+    kx = wl.k_new[sel].contiguous().view(torch.int16).cpu().numpy().view(np.uint16)
+    vx = wl.kv_new[sel].contiguous().view(torch.int16).cpu().numpy().view(np.uint16)
+    kslot, vslot = wl.k_slots[sel].cpu().numpy(), wl.kv_slots[sel].cpu().numpy()
+    t0 = time.perf_counter()
+    O.cache_store(kx, O.BF16, kslot, kd, O.E4M3, ks)
+    O.cache_store(vx, O.BF16, vslot, vd, O.E4M3, vs)
+    dt = time.perf_counter() - t0
+    return {"value": round(len(sel) / dt, 1), "unit": "tokens/s", "cores": 1, "kind": "oracle",
+            "sample": f"{len(sel)} of {n} tokens of {wl.spec.name} (key + KV rows), {dt:.2f} s"}
+
+
 # ----------------------------------------------------------------------------- oracle arm
 def _oracle_rows(wl, mode, rows):
     sys.path.insert(0, os.path.join(ROOT, "tests"))
@@ -471,8 +605,10 @@ def run_reference(args, rank, world):
     import numpy as np
     from oracle import oracle as O
     spec_fn, mode = WORKLOADS[args.workload]
-    spec = spec_fn()
     dev = "cuda" if torch.cuda.is_available() else "cpu"
+    if mode == "store":
+        return _store_reference(args, world, dev)
+    spec = spec_fn()
     wl = W.make(spec, device=dev)
     T = spec.total_q
     # size each step's sample so the whole run stays within a few minutes
@@ -504,6 +640,28 @@ def run_reference(args, rank, world):
         "cpu_baseline": {"kind": "oracle", "cores": threads, "sample": sample,
                          "value": round(value, 3), "unit": "tokens/s"},
         "e2e": {"value": round(value, 3), "unit": "tokens/s", "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }
+
+
+def _store_reference(args, world, dev):
+    wl = W.make_store(W.store_prompt_128k(), device=dev)
+    for _ in range(args.warmup):
+        _store_oracle(wl, 0, rows=2048)
+    res = [_store_oracle(wl, 0, rows=2048) for _ in range(args.steps)]
+    value = statistics.mean(r["value"] for r in res)
+    ms = 2048 / value * 1e3
+    return {
+        "impl": "reference", "metric": "cache-write tokens/s (indexer key + latent KV into FP8 "
+        "caches) on 1 B200", "value": round(value, 1), "unit": "tokens/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms, 3),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f32",
+        "data": "synthetic (seeded N(0,1) rows, 1% x4)",
+        "config": {"workload": wl.spec.name, "mode": "store", "tokens": wl.spec.n_tokens},
+        "cpu_baseline": {"kind": "oracle", "cores": 1, "value": round(value, 1),
+                         "unit": "tokens/s",
+                         "sample": f"2048 of {wl.spec.n_tokens} tokens per step (key + KV)"},
+        "e2e": {"value": round(value, 1), "unit": "tokens/s", "h2d_bytes_per_step": 0,
                 "d2h_bytes_per_step": 0},
     }
 

@@ -80,7 +80,8 @@ typedef enum dsa_dtype {
 
 /* Device check codes (dsa_device_check). */
 #define DSA_CHECK_NONE 0
-#define DSA_CHECK_BAD_PAGE 1         /* block-table entry outside [0, num_pages) */
+#define DSA_CHECK_BAD_PAGE 1         /* block-table entry outside [0, num_pages), or a
+                                        cache_store slot outside [0, num_rows) */
 #define DSA_CHECK_BAD_INDEX 2        /* top-k index outside [-1, pos] */
 #define DSA_CHECK_BAD_BATCH 3        /* nq_b > seq_lens[b], seq_lens[b] > max_seq_len, ... */
 #define DSA_CHECK_TIMEOUT 4          /* a bounded on-chip wait gave up */
@@ -228,6 +229,36 @@ DSA_API dsa_status_t dsa_decode(const void* q_idx, dsa_dtype_t q_idx_dtype,
                                 const dsa_batch_t* batch, int32_t* idx_out, void* out,
                                 dsa_dtype_t out_dtype, float* lse, void* workspace,
                                 size_t workspace_bytes, dsa_stream_t stream);
+
+/*
+ * dsa_cache_store -- writes n new tokens into a cache, the step before the
+ * indexer and the attention read them: the indexer key cache (page size 64,
+ * FP8 with a per-token key scale) and the latent-KV cache (page size 1, BF16
+ * or FP8 with a per-token scale).  Sources: "SGLang Day-0 support for
+ * DeepSeek-V3.2", section "DeepSeek Sparse Attention" (the key & key_scale
+ * cache, the token-level cache) and section "Future work" (FP8 KV cache);
+ * "DeepSeek-V3.2-Exp DSA deployment guide", section 3.1 (fp8_e4m3 KV cache).
+ *   x             [n][dim] of x_dtype (DSA_F32 or DSA_BF16), row-major
+ *   slot_mapping  [n] int64: the cache row of token i, i.e. physical page *
+ *                 page_size + position within the page (for a dsa_paged_cache_t:
+ *                 block_table[b][s / page_size] * page_size + s % page_size);
+ *                 a negative entry skips token i
+ *   cache_data    [num_rows][dim] of cache_dtype -- the page array of a cache
+ *                 seen as num_pages * page_size rows
+ *   cache_scale   [num_rows] fp32, written for an FP8 cache; ignored (may be
+ *                 NULL) for BF16 / F32 caches
+ * FP8 cache: scale = amax / 448 in fp32 with amax = max |x_e| of the row (1 for
+ * an all-zero row), code_e = e4m3(x_e / scale): the quotient is an IEEE fp32
+ * division, rounded to e4m3 to nearest even and saturated at +-448.  BF16
+ * cache: x rounded to nearest even.  F32 cache: x widened exactly.
+ * dim must be a multiple of 16 in [16, 1024]; pointers 16-byte aligned
+ * (slot_mapping 8, cache_scale 4).  A slot >= num_rows is skipped and recorded
+ * as DSA_CHECK_BAD_PAGE.  Two tokens with the same slot race (either may win).
+ */
+DSA_API dsa_status_t dsa_cache_store(const void* x, dsa_dtype_t x_dtype, int32_t n, int32_t dim,
+                                     const int64_t* slot_mapping, void* cache_data,
+                                     dsa_dtype_t cache_dtype, float* cache_scale, int64_t num_rows,
+                                     dsa_stream_t stream);
 
 /* Synchronises `stream`, then reads the current device's check word into *code
  * (a DSA_CHECK_* value, 0 if nothing was recorded) and clears it if `reset`.

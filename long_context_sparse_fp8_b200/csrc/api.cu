@@ -448,6 +448,36 @@ DSA_API dsa_status_t dsa_decode(const void* q_idx, dsa_dtype_t q_idx_dtype,
     return e == cudaSuccess ? ok() : cuda_fail(e, "decode launch");
 }
 
+DSA_API dsa_status_t dsa_cache_store(const void* x, dsa_dtype_t x_dtype, int32_t n, int32_t dim,
+                                     const int64_t* slot_mapping, void* cache_data,
+                                     dsa_dtype_t cache_dtype, float* cache_scale, int64_t num_rows,
+                                     dsa_stream_t stream) {
+    if (n < 0) return fail(DSA_ERR_INVALID_ARGUMENT, "n must be >= 0");
+    if (n == 0) return ok();
+    if (x_dtype != DSA_F32 && x_dtype != DSA_BF16)
+        return fail(valid_dtype(x_dtype) ? DSA_ERR_UNSUPPORTED : DSA_ERR_INVALID_ARGUMENT,
+                    "x_dtype must be DSA_F32 or DSA_BF16");
+    if (!valid_dtype(cache_dtype))
+        return fail(DSA_ERR_INVALID_ARGUMENT, "cache_dtype is not a dsa_dtype_t");
+    if (dim < 16 || dim > 1024 || dim % 16 != 0)
+        return fail(DSA_ERR_UNSUPPORTED, "dim (%d) must be a multiple of 16 in [16, 1024]", dim);
+    if (num_rows < 1) return fail(DSA_ERR_INVALID_ARGUMENT, "num_rows must be >= 1");
+    if (!x || !aligned16(x)) return fail(DSA_ERR_INVALID_ARGUMENT, "x must be non-NULL, 16-byte aligned");
+    if (!slot_mapping || (reinterpret_cast<uintptr_t>(slot_mapping) & 7u))
+        return fail(DSA_ERR_INVALID_ARGUMENT, "slot_mapping must be non-NULL, 8-byte aligned");
+    if (!cache_data || !aligned16(cache_data))
+        return fail(DSA_ERR_INVALID_ARGUMENT, "cache_data must be non-NULL, 16-byte aligned");
+    if (cache_dtype == DSA_FP8_E4M3 && (!cache_scale || !aligned4(cache_scale)))
+        return fail(DSA_ERR_INVALID_ARGUMENT, "an FP8 cache needs a 4-byte aligned cache_scale");
+    int* check = nullptr;
+    cudaError_t e = check_word(&check);
+    if (e == cudaSuccess)
+        e = launch_cache_store(x, x_dtype, n, dim, reinterpret_cast<const long long*>(slot_mapping),
+                               cache_data, cache_dtype, cache_scale, num_rows, check,
+                               static_cast<cudaStream_t>(stream));
+    return e == cudaSuccess ? ok() : cuda_fail(e, "cache store launch");
+}
+
 DSA_API dsa_status_t dsa_device_check(dsa_stream_t stream, int32_t* code, int32_t reset) {
     cudaError_t e = cudaStreamSynchronize(static_cast<cudaStream_t>(stream));
     if (e != cudaSuccess) return cuda_fail(e, "cudaStreamSynchronize");

@@ -48,6 +48,12 @@ cudaError_t launch_indexer_fp8_tc(const void* q, const float* q_scale, const flo
                                   const CacheView& k, const BatchView& bv, float* logits,
                                   long long ld, int* check, cudaStream_t st, bool pdl = false);
 
+// Writes n token rows of x (fp32 or bf16, [n][dim], dim % 16 == 0, dim <= 1024) into
+// cache rows slots[i] (negative: skipped) as fp8 e4m3 + amax/448 scale, bf16 or fp32.
+cudaError_t launch_cache_store(const void* x, int x_dtype, int n, int dim, const long long* slots,
+                               void* data, int cache_dtype, float* scale, long long num_rows,
+                               int* check, cudaStream_t st);
+
 // Per-row top-k by radix select.
 cudaError_t launch_topk(const float* logits, long long ld, const BatchView& bv, int k, int* idx,
                         int* check, cudaStream_t st, bool pdl = false);

@@ -31,6 +31,7 @@ EXPORTED = (
     "dsa_indexer_logits", "dsa_topk", "dsa_sparse_mla_prefill",
     "dsa_sparse_mla_decode_workspace_size", "dsa_sparse_mla_decode",
     "dsa_sparse_mla_decode_noalloc",
+    "dsa_cache_store",
     "dsa_decode_workspace_size", "dsa_decode", "dsa_device_check", "dsa_last_error_message",
     "dsa_status_string", "dsa_version",
 )
@@ -85,6 +86,8 @@ def load_library(path: str = _LIB_PATH) -> ctypes.CDLL:
         "dsa_decode_workspace_size": ([BP, i32, i32, i32], sz),
         "dsa_decode": ([P, ctypes.c_int, P, P, i32, i32, CP, i32, P, ctypes.c_int, i32, i32, i32,
                         f32, CP, BP, P, P, ctypes.c_int, P, P, sz, P], ctypes.c_int),
+        "dsa_cache_store": ([P, ctypes.c_int, i32, i32, P, P, ctypes.c_int, P, i64, P],
+                            ctypes.c_int),
         "dsa_device_check": ([P, ctypes.POINTER(i32), i32], ctypes.c_int),
         "dsa_last_error_message": ([], ctypes.c_char_p),
         "dsa_status_string": ([ctypes.c_int], ctypes.c_char_p),
@@ -233,6 +236,19 @@ def dsa_decode(q_idx, q_idx_scale, w, k_cache: PagedCache, k: int, q, kv: PagedC
         float(softmax_scale), ctypes.byref(vc), ctypes.byref(bc), _ptr(idx_out), _ptr(out),
         dtype_code(out), _ptr(lse), _ptr(workspace), ws_bytes, _stream(stream)))
     return out
+
+
+def dsa_cache_store(x, slot_mapping, cache_data, cache_scale=None, stream=None):
+    """Writes the rows of ``x`` [n, dim] (fp32 / bf16) into ``cache_data`` (any shape
+    whose last dim is ``dim``: [pages, page_size, dim] or [rows, dim]; fp8 e4m3, bf16
+    or fp32) at flat rows ``slot_mapping`` [n] int64 (negative: skipped); an fp8 cache
+    also gets its per-token ``cache_scale`` (amax / 448)."""
+    n, dim = int(x.shape[0]), int(x.shape[-1])
+    num_rows = cache_data.numel() // dim
+    _check(load_library().dsa_cache_store(
+        _ptr(x), dtype_code(x), n, dim, _ptr(slot_mapping), _ptr(cache_data),
+        dtype_code(cache_data), _ptr(cache_scale), int(num_rows), _stream(stream)))
+    return cache_data
 
 
 def dsa_device_check(reset: bool = True, stream=None) -> int:

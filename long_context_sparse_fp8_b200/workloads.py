@@ -247,3 +247,79 @@ CONFIGS = {
     4: decode_b64_128k,
     5: chunked_prefill_128k,
 }
+
+
+# ----------------------------------------------------------------------------------------
+# Cache writes: new tokens' indexer keys and latent-KV rows, and where they go.
+
+@dataclass
+class StoreSpec:
+    """New tokens to write into the two caches: ``n_tokens`` positions 0..n-1 of one
+    sequence, their page-64 key rows and page-1 KV slots drawn through seeded
+    permutations (a fragmented cache, as after many requests come and go)."""
+    name: str
+    n_tokens: int
+    idx_dim: int = 128
+    d_qk: int = 576
+    kv_fp8: bool = True            # else a bf16 KV cache
+    x_dtype: str = "bf16"          # the new rows' dtype: "bf16" | "f32"
+    spare_pages: int = 2           # cache pages / slots that receive nothing
+    skip_every: int = 0            # every skip_every-th token has slot -1 (padding)
+    heavy_frac: float = 0.01
+    heavy_mult: float = 4.0
+    seed: int = 1240
+
+
+@dataclass
+class StoreWorkload:
+    spec: StoreSpec
+    k_new: torch.Tensor            # [n, idx_dim]
+    kv_new: torch.Tensor           # [n, d_qk]
+    k_slots: torch.Tensor          # [n] int64: physical page * 64 + row, or -1
+    kv_slots: torch.Tensor         # [n] int64 slot, or -1
+    k_pages: torch.Tensor          # [pages, 64, idx_dim] fp8, pre-filled with a marker code
+    k_scale: torch.Tensor          # [pages, 64] fp32, pre-filled with -1
+    kv: torch.Tensor               # [slots, d_qk] fp8 or bf16, pre-filled with a marker
+    kv_scale: Optional[torch.Tensor]
+
+
+def make_store(spec: StoreSpec, device="cpu") -> StoreWorkload:
+    device = torch.device(device)
+    g_cpu = torch.Generator().manual_seed(spec.seed)
+    g = torch.Generator(device=device).manual_seed(spec.seed + 1)
+    n = spec.n_tokens
+    xdt = torch.bfloat16 if spec.x_dtype == "bf16" else torch.float32
+    k_new = torch.randn(n, spec.idx_dim, generator=g, device=device)
+    kv_new = torch.randn(n, spec.d_qk, generator=g, device=device)
+    n_h = int(round(spec.heavy_frac * n))
+    if n_h:
+        h = torch.randperm(n, generator=g_cpu)[:n_h].to(device)
+        k_new[h] *= spec.heavy_mult
+        kv_new[h] *= spec.heavy_mult
+    pages = (n + INDEXER_PAGE - 1) // INDEXER_PAGE + spec.spare_pages
+    page_of = torch.randperm(pages, generator=g_cpu)
+    pos = torch.arange(n)
+    k_slots = page_of[pos // INDEXER_PAGE].long() * INDEXER_PAGE + pos % INDEXER_PAGE
+    n_slots = n + spec.spare_pages * INDEXER_PAGE
+    kv_slots = torch.randperm(n_slots, generator=g_cpu)[:n].long()
+    if spec.skip_every:
+        k_slots[::spec.skip_every] = -1
+        kv_slots[::spec.skip_every] = -1
+    k_pages = torch.full((pages, INDEXER_PAGE, spec.idx_dim), 0x5A, dtype=torch.uint8,
+                         device=device).view(FP8)
+    k_scale = torch.full((pages, INDEXER_PAGE), -1.0, device=device)
+    if spec.kv_fp8:
+        kv = torch.full((n_slots, spec.d_qk), 0x5A, dtype=torch.uint8, device=device).view(FP8)
+        kv_scale = torch.full((n_slots,), -1.0, device=device)
+    else:
+        kv = torch.full((n_slots, spec.d_qk), -3.0, dtype=torch.bfloat16, device=device)
+        kv_scale = None
+    return StoreWorkload(spec=spec, k_new=k_new.to(xdt), kv_new=kv_new.to(xdt),
+                         k_slots=k_slots.to(device), kv_slots=kv_slots.to(device),
+                         k_pages=k_pages, k_scale=k_scale, kv=kv, kv_scale=kv_scale)
+
+
+def store_prompt_128k(seed: int = 1240) -> StoreSpec:
+    """A 131072-token prompt's keys and latent KV written into FP8 caches at once
+    (bf16 rows in; page-64 key cache and page-1 KV cache, fragmented)."""
+    return StoreSpec(name="store_L131072_fp8", n_tokens=131072, seed=seed)

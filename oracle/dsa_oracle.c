@@ -34,6 +34,7 @@
  *
  * Dtype codes: 0 = fp32, 1 = bf16, 2 = fp8 e4m3 (OCP).
  */
+#include <float.h>
 #include <math.h>
 #include <stdint.h>
 #include <stdlib.h>
@@ -331,8 +332,10 @@ uint16_t oracle_f32_to_bf16(float f) {
  *                 a negative entry skips the token
  *   cache_data    [num_rows][dim] of cache_dtype; cache_scale [num_rows] fp32
  * FP8 cache: amax = max_e |x_e| (fp32), scale = amax / 448 in fp32 (1 when
- * amax = 0), code_e = e4m3(x_e / scale) with the quotient an IEEE fp32
- * division.  BF16 cache: x rounded to bf16.  FP32 cache: x as is.  The scale
+ * amax = 0); the codes use the reciprocal factor inv = 448 / amax (an fp32
+ * division, capped at the largest finite fp32 so that a zero or vanishing amax
+ * gives zero codes): code_e = e4m3(x_e * inv), the product rounded to fp32.
+ * BF16 cache: x rounded to bf16.  FP32 cache: x as is.  The scale
  * of a non-FP8 cache is left untouched.  Returns -1 (after writing the valid
  * tokens) if a slot is >= num_rows.
  */
@@ -354,10 +357,12 @@ int oracle_cache_store(const void* x, int x_dtype, int64_t n, int dim,
             for (int d = 0; d < dim; ++d)
                 if (fabsf(row[d]) > amax) amax = fabsf(row[d]);
             volatile float scale = amax > 0.0f ? amax / 448.0f : 1.0f;
+            volatile float inv = 448.0f / amax;            /* +inf when amax = 0 */
+            if (inv > FLT_MAX) inv = FLT_MAX;
             uint8_t* dst = (uint8_t*)cache_data + slot * dim;
             for (int d = 0; d < dim; ++d) {
-                volatile float quotient = row[d] / scale;
-                dst[d] = oracle_f32_to_e4m3(quotient);
+                volatile float product = row[d] * inv;
+                dst[d] = oracle_f32_to_e4m3(product);
             }
             cache_scale[slot] = scale;
         } else if (cache_dtype == OR_BF16) {

@@ -152,3 +152,32 @@ def test_status_strings():
     lib = L.load_library()
     for st in range(6):
         assert lib.dsa_status_string(st).decode().startswith("DSA_")
+
+
+@pytest.mark.parametrize("case,expect", [
+    ("neg_n", D.DSA_ERR_INVALID_ARGUMENT),
+    ("x_fp8", D.DSA_ERR_UNSUPPORTED),
+    ("dim_100", D.DSA_ERR_UNSUPPORTED),
+    ("dim_2048", D.DSA_ERR_UNSUPPORTED),
+    ("misaligned_x", D.DSA_ERR_INVALID_ARGUMENT),
+    ("null_slots", D.DSA_ERR_INVALID_ARGUMENT),
+    ("fp8_no_scale", D.DSA_ERR_INVALID_ARGUMENT),
+    ("zero_rows", D.DSA_ERR_INVALID_ARGUMENT),
+    ("bad_cache_dtype", D.DSA_ERR_INVALID_ARGUMENT),
+])
+def test_cache_store_rejects_bad_arguments(case, expect):
+    a = dict(x=FAKE, xt=D.DSA_BF16, n=4, dim=128, slots=FAKE2, data=FAKE, ct=D.DSA_FP8_E4M3,
+             scale=FAKE2, rows=256)
+    a.update({"neg_n": dict(n=-1), "x_fp8": dict(xt=D.DSA_FP8_E4M3), "dim_100": dict(dim=100),
+              "dim_2048": dict(dim=2048), "misaligned_x": dict(x=FAKE + 4),
+              "null_slots": dict(slots=None), "fp8_no_scale": dict(scale=None),
+              "zero_rows": dict(rows=0), "bad_cache_dtype": dict(ct=9)}[case])
+    st = L.load_library().dsa_cache_store(a["x"], a["xt"], a["n"], a["dim"], a["slots"], a["data"],
+                                          a["ct"], a["scale"], a["rows"], None)
+    assert st == expect, _status_msg()
+    assert _status_msg()
+
+
+def test_cache_store_empty_is_a_no_op():
+    assert L.load_library().dsa_cache_store(None, D.DSA_BF16, 0, 128, None, None,
+                                            D.DSA_FP8_E4M3, None, 1, None) == D.DSA_OK

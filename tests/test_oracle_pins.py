@@ -412,8 +412,9 @@ def _cache(num_rows, dim, dtype):
 def test_cache_store_fp8_scale_codes_and_untouched_rows():
     """scale = amax / 448; the amax element becomes +-448 exactly; every code
     decodes to x / scale within half a code step (1/16 relative, 2^-10 absolute in
-    the subnormal range); an all-zero row gets scale 1 and zero codes; rows the
-    slot mapping skips or does not name keep their bytes."""
+    the subnormal range) plus the fp32 rounding of the factor 448/amax; an all-zero
+    row gets scale 1 and zero codes; rows the slot mapping skips or does not name
+    keep their bytes."""
     g = np.random.default_rng(10)
     n, dim, rows = 40, 576, 100
     x = g.standard_normal((n, dim)).astype(np.float32)
@@ -434,7 +435,7 @@ def test_cache_store_fp8_scale_codes_and_untouched_rows():
         q = x[i] / want
         dec = np.array([O.e4m3_to_double(c) for c in data[s]])
         err = np.abs(dec - q)
-        assert np.all(err <= np.maximum(np.abs(q) / 16, 2.0 ** -10) + 1e-12), i
+        assert np.all(err <= np.maximum(np.abs(q) / 16, 2.0 ** -10) * (1 + 1e-6)), i
         if amax > 0:
             j = int(np.abs(x[i]).argmax())
             assert data[s, j] == (0xFE if x[i, j] < 0 else 0x7E)
