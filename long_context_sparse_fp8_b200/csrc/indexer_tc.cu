@@ -15,11 +15,13 @@
 // Roles: warp 0 issues TMA loads (pages through the block table into a 4-stage ring
 // of 128-byte-swizzled tiles), warp 1 allocates TMEM and issues the MMAs (double-
 // buffered accumulators), the epilogue warps drain TMEM and write the logits: one
-// warpgroup for one query row per CTA (2 CTAs per SM), two warpgroups for four rows
-// (1 CTA per SM: the accumulators fill TMEM; each warpgroup reduces two rows).
+// warpgroup for one or two query rows per CTA (2 CTAs per SM), two warpgroups for
+// three or four rows (1 CTA per SM: the accumulators fill TMEM; each warpgroup
+// reduces two rows).
 //
-// Grid: x = groups of G consecutive query rows (G = 1 for decode-like batches,
-// 4 otherwise; a group that spans sequences is processed as per-sequence runs),
+// Grid: x = groups of G consecutive query rows (G = 1 for one query per sequence,
+// 2 or 3 for multi-token decode, 4 otherwise; a group that spans sequences is
+// processed as per-sequence runs),
 // y = chunks of the key tiles, so that short batches still cover all SMs.
 #include "kernels.h"
 #include "sm100.cuh"
@@ -35,10 +37,10 @@ constexpr int kTileKeys = 128;
 constexpr int kStages = 4;
 constexpr int kTileBytes = kTileKeys * kDim;       // 16 KB
 constexpr int kRowBytes = kHeads * kDim;            // one query row: 8 KB
-// 2 producer warps + EPI epilogue warpgroups: EPI = 1 for one query row per CTA
-// (64 accumulator columns, 2 CTAs per SM), EPI = 2 for four rows (the double-
-// buffered 2 x 256-column accumulator fills TMEM: 1 CTA per SM, and each warpgroup
-// reduces two of the four rows of every tile).
+// 2 producer warps + EPI epilogue warpgroups: EPI = 1 for one or two query rows per
+// CTA (64 or 128 accumulator columns, 2 CTAs per SM), EPI = 2 for three or four rows
+// (the double-buffered accumulator fills TMEM: 1 CTA per SM, and each warpgroup
+// reduces two of the rows of every tile).
 template <int EPI>
 constexpr int threads_for() { return 64 + 128 * EPI; }
 
@@ -356,14 +358,17 @@ cudaError_t make_map(CUtensorMap* m, const void* base, unsigned long long rows, 
 cudaError_t launch_indexer_fp8_tc(const void* q, const float* q_scale, const float* w,
                                   const CacheView& k, const BatchView& bv, float* logits,
                                   long long ld, int* check, cudaStream_t st, bool pdl) {
-    const int T = bv.total_q;
-    const int G = T <= 2 * bv.num_seqs ? 1 : 4;
+    // Rows per CTA: one per sequence in decode; 2 or 3 when the batch averages that
+    // many query tokens per sequence (multi-token verify), so that each sequence's
+    // keys are read once for all its rows; 4 for prefill-sized batches.
+    const int T = bv.total_q, B = bv.num_seqs;
+    const int G = T <= B ? 1 : T <= 2 * B ? 2 : T <= 3 * B ? 3 : 4;
     const int groups = (T + G - 1) / G;
     const int tiles_max = (bv.max_seq_len + kTileKeys - 1) / kTileKeys;
     // About 4 CTAs per SM (2 resident) balance long, uneven rows; when that would
     // leave fewer than 16 key tiles per CTA, one wave of 2 CTAs per SM is used
     // instead, so that the per-CTA setup is paid once per SM slot.
-    const int target = 4 * kNumSMs, slots = 2 * kNumSMs;
+    const int target = 4 * kNumSMs, slots = (G <= 2 ? 2 : 1) * kNumSMs;
     int chunks = groups >= target / 2 ? 1 : (target + groups - 1) / groups;
     if (groups < slots && tiles_max / chunks < 16) chunks = slots / groups;
     if (chunks < 1) chunks = 1;
@@ -381,7 +386,7 @@ cudaError_t launch_indexer_fp8_tc(const void* q, const float* q_scale, const flo
     const size_t smem = 1024 + kStages * kTileBytes + (size_t)G * kRowBytes +
                         (size_t)G * kHeads * sizeof(float) + 16 * sizeof(uint64_t) + 16;
     dim3 grid(groups, chunks);
-    if (G == 1) {
+    if (G <= 2) {
         e = cudaFuncSetAttribute(indexer_fp8_tc_kernel<1>,
                                  cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
         if (e != cudaSuccess) return e;

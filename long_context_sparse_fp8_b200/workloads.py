@@ -215,6 +215,14 @@ def decode_b32_8k(seed: int = 1236) -> Spec:
                 seed=seed)
 
 
+def decode_mtp_b32_8k(nq: int = 2, seed: int = 1241) -> Spec:
+    """Multi-query decode (a verify step of multi-token prediction): 32 sequences x 8192
+    context, ``nq`` query tokens each (the last nq positions); otherwise as the
+    32 x 8192 decode."""
+    return Spec(name=f"decode_mtp{nq}_b32_ctx8192", seq_lens=[8192] * 32, nq=[nq] * 32,
+                topk=2048, seed=seed)
+
+
 def prefill_32k(seed: int = 1237) -> Spec:
     """Prefill, 1 sequence L=32768, query chunk = last 8192 tokens; 1% heavy hitters x4."""
     return Spec(name="prefill_L32768_q8192", seq_lens=[32768], nq=[8192], topk=2048,

@@ -78,6 +78,39 @@ def test_fused_decode_matches_separate_calls():
     assert torch.equal(lse, lse2)
 
 
+@pytest.mark.parametrize("nq", [2, 3, 4])
+def test_multi_query_decode(nq):
+    """Decode with nq query tokens per sequence (a multi-token-prediction verify step):
+    the fused call against the oracle on sampled rows, each later token of a sequence
+    seeing one more key."""
+    wl = _wl(f"mtp{nq}", lambda: W.decode_mtp_b32_8k(nq))
+    s = wl.spec
+    batch, kc, kv = H.lib_args(wl)
+    n = L.dsa_decode_workspace_size(batch, s.topk, s.heads, s.d_v)
+    ws = torch.empty(n, dtype=torch.uint8, device="cuda")
+    out = torch.empty(s.total_q, s.heads, s.d_v, dtype=torch.bfloat16, device="cuda")
+    lse = torch.empty(s.total_q, s.heads, device="cuda")
+    idx = torch.empty(s.total_q, s.topk, dtype=torch.int32, device="cuda")
+    L.dsa_decode(wl.q_idx, None, wl.w, kc, s.topk, wl.q, kv, batch, s.d_v, s.softmax_scale, out,
+                 lse, idx, ws)
+    torch.cuda.synchronize()
+    assert L.dsa_device_check() == 0
+    rows = np.unique(np.concatenate([H.sample_rows(s.total_q, 10, seed=20 + nq),
+                                     np.arange(nq)]))           # all tokens of sequence 0
+    pos = H.positions(wl)[rows]
+    o_logits = H.oracle_logits(wl, rows)
+    g_idx = idx.cpu().numpy()[rows]
+    # the fused call keeps its logits in the workspace; the stand-alone indexer call
+    # (same kernel) gives the scores its selection must be exact on
+    g_logits = H.run_indexer(wl).cpu().numpy()[rows]
+    H.check_logits(g_logits, o_logits, pos)
+    H.check_topk(g_idx, g_logits, o_logits, pos, s.topk)
+    o_ref, l_ref = H.oracle_mla(wl, g_idx, rows)
+    H.check_mla(out.float().cpu().numpy()[rows], lse.cpu().numpy()[rows], o_ref, l_ref,
+                H.MLA_ATOL_BF16)
+    _pipeline(wl, rows, decode=True)
+
+
 def test_prefill_32k_heavy_hitters():
     wl = _wl("c3", W.prefill_32k)
     _pipeline(wl, H.sample_rows(wl.spec.total_q, 12, seed=3))
