@@ -24,8 +24,10 @@
 // a segment's worth in one warp's share), steps 2-3 fall back to radix passes over
 // the whole row and one marking sweep.  Rows longer
 // than the bitmap capacity use a second kernel that refines over the whole row and
-// emits in two ordered sweeps.
+// emits in two ordered sweeps.  Batches of a few dozen long rows (>= 32768 keys)
+// split every row over a thread-block cluster (topk_cluster_kernel, below).
 #include "kernels.h"
+#include "sm100.cuh"
 
 namespace dsa {
 namespace {
@@ -86,6 +88,9 @@ __device__ __forceinline__ int block_excl_scan(int v, Shared& sh, int* total) {
 // The bin (of nb = 1024 or 2048, counted from the top) holding the remaining-th
 // largest key, summing `copies` histograms spaced 2048 apart; *above = keys in
 // higher bins, *count = keys in the bin.  Ends synchronised.
+__device__ __forceinline__ int scan_bins(Shared& sh, const int* local, int nb, int remaining,
+                                         int* above, int* count);
+
 __device__ __forceinline__ int find_bin(Shared& sh, const int* hist, int copies, int nb,
                                         int remaining, int* above, int* count) {
     const int tid = threadIdx.x;
@@ -98,6 +103,14 @@ __device__ __forceinline__ int find_bin(Shared& sh, const int* hist, int copies,
             for (int c = 0; c < copies; ++c) local[j] += hist[c * 2048 + bin];
         }
     }
+    return scan_bins(sh, local, nb, remaining, above, count);
+}
+
+// The scan behind find_bin: thread tid holds the counts of bins nb-1-(tid*per+j).
+__device__ __forceinline__ int scan_bins(Shared& sh, const int* local, int nb, int remaining,
+                                         int* above, int* count) {
+    const int tid = threadIdx.x;
+    const int per = nb / kThreads;
     int total;
     int run = block_excl_scan(local[0] + local[1], sh, &total);
 #pragma unroll
@@ -188,7 +201,7 @@ __device__ __forceinline__ void stage_and_histogram(const float* grow, int n, ui
 
 // Bitmap of the selected positions (ascending) -> out[0, count).
 __device__ __forceinline__ void bitmap_to_list(Shared& sh, const uint32_t* bits, int words,
-                                               int* out) {
+                                               int* out, int base = 0) {
     const int tid = threadIdx.x;
     const int wpt = (words + kThreads - 1) / kThreads;
     const int w0 = min(words, tid * wpt), w1 = min(words, w0 + wpt);
@@ -200,7 +213,7 @@ __device__ __forceinline__ void bitmap_to_list(Shared& sh, const uint32_t* bits,
         uint32_t b = bits[w];
         while (b) {
             const int bit = __ffs(b) - 1;
-            out[at++] = 32 * w + bit;
+            out[at++] = base + 32 * w + bit;
             b &= b - 1u;
         }
     }
@@ -441,12 +454,308 @@ topk_long_kernel(const float* __restrict__ logits, long long ld, BatchView bv, i
     }
 }
 
+// ---------------------------------------------------------------------------------
+// Short batches (a few dozen rows): each row is split over the C CTAs of a thread-block
+// cluster (C = 2, 4 or 8), CTA r owning the contiguous segment r of the row.  The
+// method is the one above; the three histograms that fix the threshold are summed
+// across the cluster through distributed shared memory (every thread reads its bins
+// from every CTA), the equal keys at the threshold go to the lowest positions across
+// segments in rank order, and each CTA writes its selected positions at the offset
+// given by the counts of the lower ranks.  All decisions derive from cluster-summed
+// values, so every CTA takes the same branches and the same cluster barriers.
+constexpr int kCCand = 4096;               // candidates per CTA
+constexpr int kCSeg = kCCand / kWarps;     // per-warp candidate segment
+
+struct ClusterEx {
+    int slot[2][8];                        // all-gather buffers, used alternately
+};
+
+__device__ __forceinline__ int ld_cluster_s32(uint32_t caddr) {
+    int v;
+    asm volatile("ld.shared::cluster.s32 %0, [%1];" : "=r"(v) : "r"(caddr) : "memory");
+    return v;
+}
+
+__device__ __forceinline__ void st_cluster_s32(uint32_t caddr, int v) {
+    asm volatile("st.shared::cluster.s32 [%0], %1;" ::"r"(caddr), "r"(v) : "memory");
+}
+
+// Every CTA contributes v; returns the cluster total and *before = the sum over lower
+// ranks.  Uses buffer (*use)++ & 1 (each buffer is rewritten only after a later cluster
+// barrier that every reader of its previous values has passed).
+__device__ __forceinline__ int cluster_allgather_sum(ClusterEx& ex, int v, int nrank, int rank,
+                                                     int* use, int* before) {
+    const int b = (*use)++ & 1;
+    if (threadIdx.x < nrank) st_cluster_s32(sm100::mapa(sm100::smem_u32(&ex.slot[b][rank]), threadIdx.x), v);
+    sm100::cluster_sync();
+    int tot = 0, bef = 0;
+    for (int q = 0; q < nrank; ++q) {
+        const int x = ex.slot[b][q];
+        tot += x;
+        if (q < rank) bef += x;
+    }
+    *before = bef;
+    return tot;
+}
+
+// The bin of the remaining-th largest key over the cluster-summed histogram `hist`
+// (nb bins; complete in this CTA).  Ends after every CTA has read every histogram.
+__device__ __forceinline__ int cluster_find_bin(Shared& sh, const int* hist, int nb, int nrank,
+                                                int remaining, int* above, int* count) {
+    sm100::cluster_sync();                          // every CTA's histogram is complete
+    const int per = nb / kThreads;
+    int local[2] = {0, 0};
+#pragma unroll
+    for (int j = 0; j < 2; ++j) {
+        if (j < per) {
+            const uint32_t a = sm100::smem_u32(hist + (nb - 1 - (threadIdx.x * per + j)));
+            int v[8];
+#pragma unroll
+            for (int q = 0; q < 8; ++q) v[q] = q < nrank ? ld_cluster_s32(sm100::mapa(a, q)) : 0;
+#pragma unroll
+            for (int q = 0; q < 8; ++q) local[j] += v[q];
+        }
+    }
+    const int b = scan_bins(sh, local, nb, remaining, above, count);
+    sm100::cluster_sync();                          // all reads done: hist may be reused
+    return b;
+}
+
+template <class ForEach>
+__device__ __forceinline__ void cluster_refine(Shared& sh, int* hist, ForEach for_each, int shift,
+                                               int nbits, uint32_t& prefix, uint32_t& pmask,
+                                               int& remaining, int* count, int nrank) {
+    const int nb = 1 << nbits, tid = threadIdx.x;
+    for (int i = tid; i < nb; i += kThreads) hist[i] = 0;
+    __syncthreads();
+    const uint32_t pf = prefix, pm = pmask;
+    for_each([&](uint32_t key) {
+        if ((key & pm) == pf) atomicAdd(&hist[(key >> shift) & (nb - 1)], 1);
+    });
+    __syncthreads();
+    int above;
+    const int bin = cluster_find_bin(sh, hist, nb, nrank, remaining, &above, count);
+    remaining -= above;
+    prefix |= (uint32_t)bin << shift;
+    pmask |= (uint32_t)(nb - 1) << shift;
+}
+
+__global__ void __launch_bounds__(kThreads, 1)
+topk_cluster_kernel(const float* __restrict__ logits, long long ld, BatchView bv, int k,
+                    int* __restrict__ idx, int* check, int words_cap, int stage_cap) {
+    extern __shared__ __align__(16) uint8_t dyn[];
+    int* hist = reinterpret_cast<int*>(dyn);                                   // [4][2048]
+    uint32_t* ckey = reinterpret_cast<uint32_t*>(dyn + kCopies * 2048 * 4);      // [kCCand]
+    int* cpos = reinterpret_cast<int*>(ckey + kCCand);                           // [kCCand]
+    uint32_t* bitmap = reinterpret_cast<uint32_t*>(cpos + kCCand);               // [words_cap]
+    uint32_t* eqmap = bitmap + words_cap;                                        // [words_cap]
+    uint32_t* skeys = eqmap + words_cap;                                         // [stage_cap]
+    __shared__ Shared sh;
+    __shared__ ClusterEx ex;
+
+    uint32_t nrank_u;
+    asm volatile("mov.u32 %0, %%cluster_nctarank;" : "=r"(nrank_u));
+    const int nrank = (int)nrank_u, rank = (int)sm100::cluster_ctarank();
+    const int t = blockIdx.x / nrank, tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    pdl_trigger();
+    int* out = idx + (long long)t * k;
+    const RowInfo ri = row_info(bv, t, check);
+    if (!ri.ok) {
+        if (rank == 0)
+            for (int i = tid; i < k; i += kThreads) out[i] = -1;
+        return;
+    }
+    const int n = ri.pos + 1;
+    if (n <= k) {
+        if (rank == 0)
+            for (int i = tid; i < k; i += kThreads) out[i] = i < n ? i : -1;
+        return;
+    }
+    // this CTA's segment of the row: [seg0, seg0 + sn), 32-aligned
+    const int seg = (((n + nrank - 1) / nrank) + 31) & ~31;
+    const int seg0 = min(n, rank * seg), sn = min(n, seg0 + seg) - seg0;
+    const float* grow = logits + (long long)t * ld + seg0;
+    const Row row{grow, skeys, stage_cap};
+    const int words = (sn + 31) >> 5;
+    int use = 0;
+    pdl_wait();
+
+    // ---- 1. stage + top-bit histogram, summed over the cluster ---------------------
+    for (int i = tid; i < kCopies * 2048; i += kThreads) hist[i] = 0;
+    __syncthreads();
+    stage_and_histogram(grow, sn, skeys, stage_cap, hist);
+    __syncthreads();
+    for (int b = tid; b < 2048; b += kThreads)
+        hist[b] = hist[b] + hist[2048 + b] + hist[4096 + b] + hist[6144 + b];
+    __syncthreads();
+    int n_def, n_cand;
+    const uint32_t b1 = (uint32_t)cluster_find_bin(sh, hist, 2048, nrank, k, &n_def, &n_cand);
+    int remaining = k - n_def;
+    uint32_t T;
+    int n_eq;
+    auto row_each = [&](auto f) {
+        for (int i = tid; i < sn; i += kThreads) f(row(i));
+    };
+
+    // ---- 2. bitmap of the higher bins; candidates of bin b1 into per-warp segments
+    int c_at = 0;
+    for (int g0 = warp; g0 < words; g0 += 4 * kWarps) {
+        uint32_t kk[4];
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+            const int i = 32 * (g0 + u * kWarps) + lane;
+            kk[u] = i < sn ? row(i) : 0u;
+        }
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+            const int g = g0 + u * kWarps;
+            if (g >= words) break;
+            const int i = 32 * g + lane;
+            const uint32_t bin = kk[u] >> (32 - kTopBits);
+            const unsigned md = __ballot_sync(0xffffffffu, i < sn && bin > b1);
+            const bool cand = i < sn && bin == b1;
+            const unsigned mc = __ballot_sync(0xffffffffu, cand);
+            if (lane == 0) {
+                bitmap[g] = md;
+                eqmap[g] = 0u;
+            }
+            if (mc) {
+                const int c = c_at + __popc(mc & ((1u << lane) - 1u));
+                if (cand && c < kCSeg) {
+                    ckey[warp * kCSeg + c] = kk[u] & kLowMask;
+                    cpos[warp * kCSeg + c] = i;
+                }
+                c_at += __popc(mc);
+            }
+        }
+    }
+    if (lane == 0) sh.seg_n[warp] = c_at;
+    const int over_local = __syncthreads_or(c_at > kCSeg) ? 1 : 0;
+    int dummy;
+    const bool fast = cluster_allgather_sum(ex, over_local, nrank, rank, &use, &dummy) == 0;
+
+    if (fast) {
+        // ---- 3. exact threshold among the cluster's candidates; mark them ----------
+        const int seg_cnt = sh.seg_n[warp];
+        auto cand_each = [&](auto f) {
+            for (int c = lane; c < seg_cnt; c += 32) f(ckey[warp * kCSeg + c]);
+        };
+        uint32_t prefix = 0u, pmask = 0u;
+        cluster_refine(sh, hist, cand_each, 10, 11, prefix, pmask, remaining, &n_eq, nrank);
+        cluster_refine(sh, hist, cand_each, 0, 10, prefix, pmask, remaining, &n_eq, nrank);
+        T = prefix;
+        for (int c = lane; c < seg_cnt; c += 32) {
+            const uint32_t key = ckey[warp * kCSeg + c];
+            const int p = cpos[warp * kCSeg + c];
+            if (key > T) atomicOr(&bitmap[p >> 5], 1u << (p & 31));
+            else if (key == T) atomicOr(&eqmap[p >> 5], 1u << (p & 31));
+        }
+    } else {
+        // ---- fallback: refine over the segments, then one marking sweep --------------
+        uint32_t prefix = b1 << (32 - kTopBits);
+        uint32_t pmask = ~kLowMask;
+        cluster_refine(sh, hist, row_each, 10, 11, prefix, pmask, remaining, &n_eq, nrank);
+        cluster_refine(sh, hist, row_each, 0, 10, prefix, pmask, remaining, &n_eq, nrank);
+        T = prefix;
+        for (int g0 = warp; g0 < words; g0 += kWarps) {
+            const int i = 32 * g0 + lane;
+            const uint32_t key = i < sn ? row(i) : 0u;
+            const unsigned mg = __ballot_sync(0xffffffffu, i < sn && key > T);
+            const unsigned me = __ballot_sync(0xffffffffu, i < sn && key == T);
+            if (lane == 0) {
+                bitmap[g0] = mg;
+                eqmap[g0] = me;
+            }
+        }
+    }
+    __syncthreads();
+
+    // ---- equal keys: the `remaining` lowest positions of the whole row -------------
+    {
+        const int wpt = (words + kThreads - 1) / kThreads;
+        const int w0 = min(words, tid * wpt), w1 = min(words, w0 + wpt);
+        int c = 0;
+        for (int w = w0; w < w1; ++w) c += __popc(eqmap[w]);
+        int local_eq;
+        int before = block_excl_scan(c, sh, &local_eq);
+        int eq_lower;
+        cluster_allgather_sum(ex, local_eq, nrank, rank, &use, &eq_lower);
+        const int take = max(0, min(local_eq, remaining - eq_lower));
+        for (int w = w0; w < w1 && before < take; ++w) {
+            uint32_t e = eqmap[w];
+            const int pc = __popc(e);
+            if (before + pc > take) {
+                for (int drop = before + pc - take; drop > 0; --drop)
+                    e &= ~(0x80000000u >> __clz(e));
+            }
+            bitmap[w] |= e;
+            before += pc;
+        }
+    }
+    __syncthreads();
+
+    // ---- 4. ascending output: this segment's positions after the lower ranks' -------
+    {
+        const int wpt = (words + kThreads - 1) / kThreads;
+        const int w0 = min(words, tid * wpt), w1 = min(words, w0 + wpt);
+        int c = 0;
+        for (int w = w0; w < w1; ++w) c += __popc(bitmap[w]);
+        int local_sel;
+        block_excl_scan(c, sh, &local_sel);
+        int sel_lower;
+        cluster_allgather_sum(ex, local_sel, nrank, rank, &use, &sel_lower);
+        bitmap_to_list(sh, bitmap, words, out + sel_lower, seg0);
+    }
+}
+
 }  // namespace
 
 cudaError_t launch_topk(const float* logits, long long ld, const BatchView& bv, int k, int* idx,
                         int* check, cudaStream_t st, bool pdl) {
     const int hist_bytes = kCopies * 2048 * 4;
     const int words = ((bv.max_seq_len + 31) / 32 + 3) & ~3;
+    // A few dozen long rows would leave most SMs idle with one CTA per row, and a row
+    // beyond the staging capacity is re-read from L2: split each row over a cluster of
+    // C CTAs instead.  (Rows of ~8K keys measured slower this way: the cluster barriers
+    // and exchanges cost more than the split saves.)
+    const int T = bv.total_q;
+    const int C = T <= kNumSMs / 8 ? 8 : T <= kNumSMs / 4 ? 4 : T <= kNumSMs / 2 ? 2 : 1;
+    const int cseg = (((bv.max_seq_len + C - 1) / C) + 31) & ~31;
+    if (C > 1 && bv.max_seq_len >= 32768 && bv.max_seq_len > 2 * k && cseg <= 32 * kMaxWords) {
+        const int seg = cseg;
+        const int cwords = ((seg / 32) + 3) & ~3;
+        const int fixed = hist_bytes + kCCand * 8 + 2 * cwords * 4;
+        int stage = (kSmemLimit - kStaticReserve - fixed) / 4 & ~3;
+        if (stage > seg) stage = seg;
+        const size_t smem = (size_t)fixed + (size_t)stage * 4;
+        cudaError_t e = cudaFuncSetAttribute(topk_cluster_kernel,
+                                             cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+        if (e != cudaSuccess) return e;
+        cudaLaunchConfig_t cfg = {};
+        cfg.gridDim = dim3(T * C);
+        cfg.blockDim = dim3(kThreads);
+        cfg.dynamicSmemBytes = smem;
+        cfg.stream = st;
+        cudaLaunchAttribute attr[2];
+        attr[0].id = cudaLaunchAttributeClusterDimension;
+        attr[0].val.clusterDim.x = C;
+        attr[0].val.clusterDim.y = 1;
+        attr[0].val.clusterDim.z = 1;
+        attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+        attr[1].val.programmaticStreamSerializationAllowed = 1;
+        cfg.attrs = attr;
+        cfg.numAttrs = 1;
+        int clusters = 0;
+        e = cudaOccupancyMaxActiveClusters(&clusters, topk_cluster_kernel, &cfg);
+        if (e == cudaSuccess && clusters > 0) {
+            cfg.numAttrs = pdl ? 2 : 1;
+            e = cudaLaunchKernelEx(&cfg, topk_cluster_kernel, logits, ld, bv, k, idx, check, cwords,
+                                   stage);
+            if (e != cudaSuccess) return e;
+            return cudaGetLastError();
+        }
+        (void)cudaGetLastError();   // no cluster fits: one CTA per row below
+    }
     if (words <= kMaxWords) {
         const int fixed = hist_bytes + kCandCap * 8 + 2 * words * 4;
         int stage = (kSmemLimit - kStaticReserve - fixed) / 4 & ~3;

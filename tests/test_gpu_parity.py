@@ -201,6 +201,40 @@ def test_topk_candidates_concentrated_in_one_warp():
     H.check_topk(got, logits.cpu().numpy(), logits.cpu().numpy(), np.array([n - 1]), k)
 
 
+@pytest.mark.parametrize("kind", ["normal", "coarse", "three"])
+def test_topk_cluster_split_matches_one_cta_per_row(kind):
+    """Short batches of long rows split each row over a cluster of 8, 4 or 2 CTAs;
+    larger batches give each row one CTA.  The same rows must get the same lists
+    either way (ragged lengths, so some clusters hold rows far shorter than the
+    longest)."""
+    n, k, T = 40000, 2048, 200
+    g = torch.Generator(device="cuda").manual_seed(99)
+    x = torch.randn(T, n, generator=g, device="cuda")
+    if kind == "coarse":
+        x = torch.round(x * 20) / 20
+    elif kind == "three":
+        x = torch.randint(0, 3, (T, n), generator=g, device="cuda").float()
+    lens = torch.randint(3000, n + 1, (T,), generator=g, device="cuda").to(torch.int32)
+    lens[0] = n
+    logits = x.contiguous()
+    def run(rows):
+        cu = torch.arange(rows + 1, dtype=torch.int32, device="cuda")
+        b = L.Batch(cu, lens[:rows].contiguous(), rows, n)
+        idx = torch.empty(rows, k, dtype=torch.int32, device="cuda")
+        L.dsa_topk(logits[:rows], b, k, idx)
+        torch.cuda.synchronize()
+        return idx.cpu().numpy()
+    full = run(T)                                  # one CTA per row
+    for rows in (16, 36, 72):                      # clusters of 8, 4, 2
+        part = run(rows)
+        assert np.array_equal(part, full[:rows]), rows
+    assert L.dsa_device_check() == 0
+    pos = lens.cpu().numpy() - 1
+    lg = logits.cpu().numpy()
+    sel = np.array([0, 5, 71])
+    H.check_topk(full[sel], lg[sel], lg[sel], pos[sel], k)
+
+
 def test_device_check_reports_bad_index_and_page():
     spec = W.Spec(name="chk", seq_lens=[300], nq=[4], topk=64, seed=5)
     wl = W.make(spec, device="cuda")
