@@ -16,6 +16,8 @@
 // group, the factor 448/amax is formed once per row, and each lane converts and
 // stores its chunks (8 B of e4m3 codes, 16 B of bf16 or 32 B of fp32).  HBM-bound:
 // dim x (input + output bytes) + 4 B scale + 8 B slot per token.
+#include <atomic>
+
 #include "common.cuh"
 #include "kernels.h"
 
@@ -169,13 +171,15 @@ cudaError_t launch_shape(const void* x, int n, int dim, const long long* slots, 
                          float* scale, long long num_rows, int* check, cudaStream_t st) {
     constexpr int kRowsPerBlock = (kThreads / 32) * kRowsPerGroup * (32 / LPR);
     // one wave: as many blocks as fit on the SMs at once (queried once per shape)
-    static int per_sm = 0;
+    static std::atomic<int> cached{0};
+    int per_sm = cached.load(std::memory_order_relaxed);
     if (per_sm == 0) {
         int b = 0;
         cudaError_t e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(
             &b, cache_store_kernel<XT, CT, LPR, CPL>, kThreads, 0);
         if (e != cudaSuccess) return e;
         per_sm = b > 0 ? b : 1;
+        cached.store(per_sm, std::memory_order_relaxed);
     }
     const long long blocks = ((long long)n + kRowsPerBlock - 1) / kRowsPerBlock;
     const long long wave = (long long)per_sm * kNumSMs;

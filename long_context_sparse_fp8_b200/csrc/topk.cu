@@ -26,6 +26,11 @@
 // than the bitmap capacity use a second kernel that refines over the whole row and
 // emits in two ordered sweeps.  Batches of a few dozen long rows (>= 32768 keys)
 // split every row over a thread-block cluster (topk_cluster_kernel, below).
+#include <algorithm>
+#include <mutex>
+#include <utility>
+#include <vector>
+
 #include "kernels.h"
 #include "sm100.cuh"
 
@@ -745,16 +750,34 @@ cudaError_t launch_topk(const float* logits, long long ld, const BatchView& bv, 
         attr[1].val.programmaticStreamSerializationAllowed = 1;
         cfg.attrs = attr;
         cfg.numAttrs = 1;
+        // whether a cluster of this shape fits, asked once per (C, shared memory)
         int clusters = 0;
-        e = cudaOccupancyMaxActiveClusters(&clusters, topk_cluster_kernel, &cfg);
-        if (e == cudaSuccess && clusters > 0) {
+        {
+            static std::mutex mu;
+            static std::vector<std::pair<long long, int>> known;
+            const long long key = (long long)C << 32 | (long long)smem;
+            std::lock_guard<std::mutex> lk(mu);
+            auto it = std::find_if(known.begin(), known.end(),
+                                   [&](const std::pair<long long, int>& kv) { return kv.first == key; });
+            if (it != known.end()) {
+                clusters = it->second;
+            } else {
+                e = cudaOccupancyMaxActiveClusters(&clusters, topk_cluster_kernel, &cfg);
+                if (e != cudaSuccess) {
+                    (void)cudaGetLastError();
+                    clusters = 0;
+                }
+                known.emplace_back(key, clusters);
+            }
+        }
+        if (clusters > 0) {
             cfg.numAttrs = pdl ? 2 : 1;
             e = cudaLaunchKernelEx(&cfg, topk_cluster_kernel, logits, ld, bv, k, idx, check, cwords,
                                    stage);
             if (e != cudaSuccess) return e;
             return cudaGetLastError();
         }
-        (void)cudaGetLastError();   // no cluster fits: one CTA per row below
+        // no cluster fits: one CTA per row below
     }
     if (words <= kMaxWords) {
         const int fixed = hist_bytes + kCandCap * 8 + 2 * words * 4;
