@@ -264,6 +264,18 @@ class Step:
         }
 
 
+def sparse_ratio(spec) -> float:
+    """Mean over query rows of the attended fraction of the causal keys, min(k, pos+1) /
+    (pos+1) -- what a serving stack reports as its sparse-attention ratio."""
+    tot, n = 0.0, 0
+    for b in range(spec.num_seqs):
+        for i in range(spec.nq[b]):
+            pos = spec.seq_lens[b] - spec.nq[b] + i
+            tot += min(spec.topk, pos + 1) / (pos + 1)
+            n += 1
+    return round(tot / max(n, 1), 5)
+
+
 def timed_loop(fn_list, steps, flush, stream):
     """K steps; before each, a 256 MiB write flushes L2; events around every stage."""
     evs = []
@@ -434,6 +446,7 @@ def run_dsa(args, rank, world, dev):
                    "mla": f"{spec.heads} heads, d_qk {spec.d_qk}, d_v {spec.d_v}, "
                           f"{'fp8' if spec.kv_fp8 else 'bf16'} latent KV page 1",
                    "l2": "flushed between steps (256 MiB write)",
+                   "sparse_attention_ratio": sparse_ratio(spec),
                    "parallelism": f"replicas x{world}"},
         "roofline": roof, "cpu_baseline": cpu, "e2e": e2e, "clocks": clk.summary(),
         "gpu_launches": st.launches_per_step() * args.steps,

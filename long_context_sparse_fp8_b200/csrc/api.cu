@@ -6,6 +6,8 @@
 #include <mutex>
 #include <string>
 
+#include <nvtx3/nvToolsExt.h>
+
 #include "dsa.h"
 #include "kernels.h"
 
@@ -14,6 +16,13 @@ namespace {
 using namespace dsa;
 
 thread_local std::string g_msg;
+
+// An NVTX range around each entry point (visible in Nsight timelines; a no-op when no
+// tool is attached).
+struct Range {
+    explicit Range(const char* name) { nvtxRangePushA(name); }
+    ~Range() { nvtxRangePop(); }
+};
 
 dsa_status_t fail(dsa_status_t st, const char* fmt, ...) {
     char buf[512];
@@ -266,6 +275,7 @@ DSA_API dsa_status_t dsa_indexer_logits(const void* q, dsa_dtype_t q_dtype, cons
                                         const float* w, int32_t heads, int32_t dim,
                                         const dsa_paged_cache_t* k_cache, const dsa_batch_t* batch,
                                         float* logits, int64_t ld_logits, dsa_stream_t stream) {
+    Range nvtx_range("dsa_indexer_logits");
     BatchView bv;
     CacheView kc;
     dsa_status_t s = check_batch(batch, &bv);
@@ -283,6 +293,7 @@ DSA_API dsa_status_t dsa_indexer_logits(const void* q, dsa_dtype_t q_dtype, cons
 
 DSA_API dsa_status_t dsa_topk(const float* logits, int64_t ld_logits, const dsa_batch_t* batch,
                               int32_t k, int32_t* idx, dsa_stream_t stream) {
+    Range nvtx_range("dsa_topk");
     BatchView bv;
     dsa_status_t s = check_batch(batch, &bv);
     if (s != DSA_OK || bv.total_q == 0) return s == DSA_OK ? ok() : s;
@@ -301,6 +312,7 @@ DSA_API dsa_status_t dsa_sparse_mla_prefill(const void* q, dsa_dtype_t q_dtype, 
                                             const dsa_paged_cache_t* kv, const dsa_batch_t* batch,
                                             const int32_t* idx, int32_t k, void* out,
                                             dsa_dtype_t out_dtype, float* lse, dsa_stream_t stream) {
+    Range nvtx_range("dsa_sparse_mla_prefill");
     BatchView bv;
     MlaPlan plan;
     dsa_status_t s = check_batch(batch, &bv);
@@ -329,6 +341,7 @@ DSA_API dsa_status_t dsa_sparse_mla_decode(const void* q, dsa_dtype_t q_dtype, i
                                            const int32_t* idx, int32_t k, void* out,
                                            dsa_dtype_t out_dtype, float* lse, void* workspace,
                                            size_t workspace_bytes, dsa_stream_t stream) {
+    Range nvtx_range("dsa_sparse_mla_decode");
     BatchView bv;
     MlaPlan plan;
     dsa_status_t s = check_batch(batch, &bv);
@@ -352,6 +365,7 @@ DSA_API dsa_status_t dsa_sparse_mla_decode_noalloc(const void* q, dsa_dtype_t q_
                                                    const dsa_batch_t* batch, const int32_t* idx,
                                                    int32_t k, void* out, dsa_dtype_t out_dtype,
                                                    float* lse, dsa_stream_t stream) {
+    Range nvtx_range("dsa_sparse_mla_decode_noalloc");
     static_assert(kStaticScratchBytes == DSA_NOALLOC_SCRATCH_BYTES, "scratch size mismatch");
     BatchView bv;
     MlaPlan plan;
@@ -397,6 +411,7 @@ DSA_API dsa_status_t dsa_decode(const void* q_idx, dsa_dtype_t q_idx_dtype,
                                 const dsa_batch_t* batch, int32_t* idx_out, void* out,
                                 dsa_dtype_t out_dtype, float* lse, void* workspace,
                                 size_t workspace_bytes, dsa_stream_t stream) {
+    Range nvtx_range("dsa_decode");
     BatchView bv;
     dsa_status_t s = check_batch(batch, &bv);
     if (s != DSA_OK || bv.total_q == 0) return s == DSA_OK ? ok() : s;
@@ -452,6 +467,7 @@ DSA_API dsa_status_t dsa_cache_store(const void* x, dsa_dtype_t x_dtype, int32_t
                                      const int64_t* slot_mapping, void* cache_data,
                                      dsa_dtype_t cache_dtype, float* cache_scale, int64_t num_rows,
                                      dsa_stream_t stream) {
+    Range nvtx_range("dsa_cache_store");
     if (n < 0) return fail(DSA_ERR_INVALID_ARGUMENT, "n must be >= 0");
     if (n == 0) return ok();
     if (x_dtype != DSA_F32 && x_dtype != DSA_BF16)
@@ -479,6 +495,7 @@ DSA_API dsa_status_t dsa_cache_store(const void* x, dsa_dtype_t x_dtype, int32_t
 }
 
 DSA_API dsa_status_t dsa_device_check(dsa_stream_t stream, int32_t* code, int32_t reset) {
+    Range nvtx_range("dsa_device_check");
     cudaError_t e = cudaStreamSynchronize(static_cast<cudaStream_t>(stream));
     if (e != cudaSuccess) return cuda_fail(e, "cudaStreamSynchronize");
     int v = 0;
