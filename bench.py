@@ -341,6 +341,22 @@ def run_dsa(args, rank, world, dev):
     roof["peak_source"] = f"{peak_kind} ({'burst' if roof['unit'] == 'GB/s' else 'burst bf16'})"
     roof["stage_ms"] = {n: round(v, 4) for n, v in mean_stage.items()}
     roof["algorithmic_bytes_per_launch"] = work[dom]["bytes"]
+    if mode == "prefill":
+        # the same selection without the [T][L] logits: dsa_indexer_topk over L2-sized
+        # row blocks (reported beside the staged calls the step uses)
+        ws_n = L.dsa_indexer_topk_workspace_size(st.batch)
+        ws_fused = torch.empty(max(ws_n, 16), dtype=torch.uint8, device=dev)
+        idx_f = torch.empty_like(st.idx)
+        fused_call = lambda: L.dsa_indexer_topk(wl.q_idx, None, wl.w, st.kc, st.batch,  # noqa: E731
+                                                spec.topk, idx_f, workspace=ws_fused)
+        for _ in range(2):
+            fused_call()
+        R.barrier(world, dev)
+        f_ms = statistics.mean(r[0] for r in timed_loop([fused_call], args.steps, flush, stream))
+        roof["indexer_topk_fused"] = {
+            "ms": round(f_ms, 4), "staged_ms": round(mean_stage["indexer"] + mean_stage["topk"], 4),
+            "logits_bytes_staged": int(st.logits.numel() * 4), "logits_bytes_fused": int(ws_n),
+            "same_selection": bool(torch.equal(idx_f, st.idx))}
 
     # ---- end to end through host buffers: every step uploads its queries (q_idx, w, q)
     # from pinned host memory and downloads o, as a serving loop does -- the uploads of

@@ -231,6 +231,25 @@ DSA_API dsa_status_t dsa_decode(const void* q_idx, dsa_dtype_t q_idx_dtype,
                                 size_t workspace_bytes, dsa_stream_t stream);
 
 /*
+ * dsa_indexer_topk -- the indexer and the top-k without the full logits matrix
+ * ("SGLang Day-0 support for DeepSeek-V3.2", its launch lines' FUSE_TOPK switch: the
+ * selection fused with the scoring).  The query rows are processed in blocks whose
+ * logits take at most 80 MB of the L2 (592 rows at 32K context, 160 at 128K); each
+ * block's logits go to the workspace and are selected from at once, so they do not
+ * round-trip through HBM and the memory needed is one block, not [T][L].
+ * Arguments and results are those of dsa_indexer_logits followed by dsa_topk
+ * (idx [T][k]: identical lists); workspace: dsa_indexer_topk_workspace_size bytes,
+ * 16-byte aligned, contents undefined afterwards.  Meant for prefill-sized batches;
+ * for decode, dsa_decode keeps the whole step in one call.
+ */
+DSA_API size_t dsa_indexer_topk_workspace_size(const dsa_batch_t* batch);
+DSA_API dsa_status_t dsa_indexer_topk(const void* q, dsa_dtype_t q_dtype, const float* q_scale,
+                                      const float* w, int32_t heads, int32_t dim,
+                                      const dsa_paged_cache_t* k_cache, const dsa_batch_t* batch,
+                                      int32_t k, int32_t* idx, void* workspace,
+                                      size_t workspace_bytes, dsa_stream_t stream);
+
+/*
  * dsa_cache_store -- writes n new tokens into a cache, the step before the
  * indexer and the attention read them: the indexer key cache (page size 64,
  * FP8 with a per-token key scale) and the latent-KV cache (page size 1, BF16

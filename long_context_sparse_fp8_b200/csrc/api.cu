@@ -141,10 +141,10 @@ dsa_status_t indexer_validate(const void* q, dsa_dtype_t q_dtype, const float* q
 
 cudaError_t indexer_launch(const void* q, const float* q_scale, const float* w, int heads, int dim,
                            const CacheView& kc, const BatchView& bv, float* logits, long long ld,
-                           int* check, cudaStream_t st, bool pdl = false) {
+                           int* check, cudaStream_t st, bool pdl = false, int row0 = 0) {
     if (kc.dtype == kE4M3)  // validated: 64 heads x 128 dims
-        return launch_indexer_fp8_tc(q, q_scale, w, kc, bv, logits, ld, check, st, pdl);
-    return launch_indexer_generic(q, q_scale, w, heads, dim, kc, bv, logits, ld, check, st);
+        return launch_indexer_fp8_tc(q, q_scale, w, kc, bv, logits, ld, check, st, pdl, row0);
+    return launch_indexer_generic(q, q_scale, w, heads, dim, kc, bv, logits, ld, check, st, row0);
 }
 
 // ---------------------------------------------------------------- top-k
@@ -461,6 +461,65 @@ DSA_API dsa_status_t dsa_decode(const void* q_idx, dsa_dtype_t q_idx_dtype,
         e = mla_decode_launch(plan, q, heads, d_qk, d_v, softmax_scale, bv, sel, k, out, out_dtype,
                               lse, mla_ws, check, st, true);
     return e == cudaSuccess ? ok() : cuda_fail(e, "decode launch");
+}
+
+// Rows per block of dsa_indexer_topk: the logits of one block take at most 80 MB of the
+// 126 MB L2, so the top-k reads them while they are still on chip; where that allows
+// several hundred rows, a multiple of 592 (4 rows per indexer CTA x 148 SMs, and one
+// top-k CTA per row) so that both kernels run whole waves.
+constexpr size_t kL2BlockBytes = (size_t)80 << 20;
+constexpr int kWaveRows = 4 * kNumSMs;
+
+int indexer_topk_block_rows(int total_q, long long ld) {
+    long long rows = (long long)(kL2BlockBytes / ((size_t)ld * sizeof(float)));
+    rows = rows >= kWaveRows ? rows / kWaveRows * kWaveRows : rows & ~3LL;
+    if (rows < 4) rows = 4;
+    if (rows > total_q) rows = total_q;
+    return (int)rows;
+}
+
+DSA_API size_t dsa_indexer_topk_workspace_size(const dsa_batch_t* batch) {
+    if (!batch || batch->total_q < 0 || batch->max_seq_len < 1) return 0;
+    const long long ld = decode_ld(batch->max_seq_len);
+    const int rows = indexer_topk_block_rows(batch->total_q, ld);
+    return align_up((size_t)(rows > 0 ? rows : 0) * (size_t)ld * sizeof(float), 256);
+}
+
+DSA_API dsa_status_t dsa_indexer_topk(const void* q, dsa_dtype_t q_dtype, const float* q_scale,
+                                      const float* w, int32_t heads, int32_t dim,
+                                      const dsa_paged_cache_t* k_cache, const dsa_batch_t* batch,
+                                      int32_t k, int32_t* idx, void* workspace,
+                                      size_t workspace_bytes, dsa_stream_t stream) {
+    Range nvtx_range("dsa_indexer_topk");
+    BatchView bv;
+    dsa_status_t s = check_batch(batch, &bv);
+    if (s != DSA_OK || bv.total_q == 0) return s == DSA_OK ? ok() : s;
+    if (!workspace || !aligned16(workspace))
+        return fail(DSA_ERR_INVALID_ARGUMENT, "workspace must be non-NULL and 16-byte aligned");
+    const size_t need = dsa_indexer_topk_workspace_size(batch);
+    if (workspace_bytes < need)
+        return fail(DSA_ERR_WORKSPACE_TOO_SMALL, "workspace needs %zu bytes, got %zu", need,
+                    workspace_bytes);
+    const long long ld = decode_ld(bv.max_seq_len);
+    float* logits = static_cast<float*>(workspace);
+    CacheView kc;
+    s = indexer_validate(q, q_dtype, q_scale, w, heads, dim, k_cache, bv, logits, ld, &kc);
+    if (s == DSA_OK) s = topk_validate(logits, ld, bv, k, idx);
+    if (s != DSA_OK) return s;
+    int* check = nullptr;
+    cudaError_t e = check_word(&check);
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    // Blocks of rows: the indexer writes a block's logits, the top-k selects from them
+    // (programmatic dependents; each kernel waits for its predecessor before touching
+    // the shared buffer, so block i+1's logits never overwrite what block i still reads).
+    const int rows = indexer_topk_block_rows(bv.total_q, ld);
+    for (int r0 = 0; e == cudaSuccess && r0 < bv.total_q; r0 += rows) {
+        BatchView blk = bv;
+        blk.total_q = r0 + rows < bv.total_q ? r0 + rows : bv.total_q;
+        e = indexer_launch(q, q_scale, w, heads, dim, kc, blk, logits, ld, check, st, true, r0);
+        if (e == cudaSuccess) e = launch_topk(logits, ld, blk, k, idx, check, st, true, r0);
+    }
+    return e == cudaSuccess ? ok() : cuda_fail(e, "indexer + top-k launch");
 }
 
 DSA_API dsa_status_t dsa_cache_store(const void* x, dsa_dtype_t x_dtype, int32_t n, int32_t dim,

@@ -18,9 +18,10 @@ template <int DT>
 __global__ void __launch_bounds__(kThreads)
 indexer_generic_kernel(const void* __restrict__ q, const float* __restrict__ q_scale,
                        const float* __restrict__ w, int heads, int dim, CacheView kc, BatchView bv,
-                       float* __restrict__ logits, long long ld, int* check) {
+                       float* __restrict__ logits, long long ld, int row0, int* check) {
     extern __shared__ float sm[];
-    const int t = blockIdx.x, tile = blockIdx.y, tid = threadIdx.x;
+    const int t = row0 + blockIdx.x, tile = blockIdx.y, tid = threadIdx.x;
+    logits -= (long long)row0 * ld;          // row t of the launch is logits row t - row0
     const RowInfo ri = row_info(bv, t, check);
     if (!ri.ok) return;
     const int s0 = tile * kIndexerPage;
@@ -76,15 +77,15 @@ indexer_generic_kernel(const void* __restrict__ q, const float* __restrict__ q_s
 
 cudaError_t launch_indexer_generic(const void* q, const float* q_scale, const float* w, int heads,
                                    int dim, const CacheView& k, const BatchView& bv, float* logits,
-                                   long long ld, int* check, cudaStream_t st) {
+                                   long long ld, int* check, cudaStream_t st, int row0) {
     const int tiles = (bv.max_seq_len + kIndexerPage - 1) / kIndexerPage;
     const size_t smem = sizeof(float) * ((size_t)(heads + kIndexerPage) * (dim + 1) + heads + 64);
     auto kern = k.dtype == kE4M3 ? indexer_generic_kernel<kE4M3> : indexer_generic_kernel<kF32>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          (int)smem);
     if (e != cudaSuccess) return e;
-    dim3 grid(bv.total_q, tiles);
-    kern<<<grid, kThreads, smem, st>>>(q, q_scale, w, heads, dim, k, bv, logits, ld, check);
+    dim3 grid(bv.total_q - row0, tiles);
+    kern<<<grid, kThreads, smem, st>>>(q, q_scale, w, heads, dim, k, bv, logits, ld, row0, check);
     return cudaGetLastError();
 }
 

@@ -56,6 +56,7 @@ struct Params {
     long long ld;
     int G;          // query rows per CTA
     int C;          // key tiles per chunk
+    int row0;       // first query row of the launch; logits row t is at (t - row0) * ld
     int* check;
 };
 
@@ -66,7 +67,7 @@ struct Run {        // a run of query rows of one sequence (j0 == j1: nothing to
 // The r-th per-sequence run of the CTA's row group, restricted to its key chunk.
 // Returns false when there is no such run.
 __device__ __forceinline__ bool get_run(const Params& p, int k, Run* out, bool skip) {
-    const int t_begin = blockIdx.x * p.G;
+    const int t_begin = p.row0 + blockIdx.x * p.G;
     const int t_end = min(p.bv.total_q, t_begin + p.G);
     int t = t_begin;
     for (int i = 0; t < t_end; ++i) {
@@ -141,7 +142,7 @@ indexer_fp8_tc_kernel(const __grid_constant__ CUtensorMap tm_k,
     }
     pdl_wait();   // launched as a dependent: every input may come from the previous kernel
     {   // head weights of the CTA's rows, loaded once (no per-run barrier needed)
-        const int t_begin = blockIdx.x * p.G;
+        const int t_begin = p.row0 + blockIdx.x * p.G;
         const int nrow = min(p.G, p.bv.total_q - t_begin);
         for (int i = threadIdx.x; i < nrow * kHeads; i += threads_for<EPI>())
             w_s[i] = __ldg(p.w + (long long)t_begin * kHeads + i);
@@ -265,7 +266,7 @@ indexer_fp8_tc_kernel(const __grid_constant__ CUtensorMap tm_k,
         Run run;
         for (int k = 0; alive && get_run(p, k, &run, skip); ++k) {
             if (run.j0 >= run.j1) continue;
-            const float* w_run = w_s + (run.t0 - blockIdx.x * p.G) * kHeads;
+            const float* w_run = w_s + (run.t0 - p.row0 - blockIdx.x * p.G) * kHeads;
             float qs[4];
 #pragma unroll
             for (int i = 0; i < 4; ++i)
@@ -333,7 +334,7 @@ indexer_fp8_tc_kernel(const __grid_constant__ CUtensorMap tm_k,
                     const int qi = q_lo + u;
                     if (qi >= run.r) break;
                     const int pos = run.pos_lo + qi;
-                    float* dst = p.logits + (long long)(run.t0 + qi) * p.ld + s;
+                    float* dst = p.logits + (long long)(run.t0 + qi - p.row0) * p.ld + s;
                     if (s <= pos) *dst = bad ? -INFINITY : res[u] * ks * qs[qi];
                     else if (s < p.ld) *dst = -INFINITY;
                 }
@@ -357,11 +358,12 @@ cudaError_t make_map(CUtensorMap* m, const void* base, unsigned long long rows, 
 
 cudaError_t launch_indexer_fp8_tc(const void* q, const float* q_scale, const float* w,
                                   const CacheView& k, const BatchView& bv, float* logits,
-                                  long long ld, int* check, cudaStream_t st, bool pdl) {
+                                  long long ld, int* check, cudaStream_t st, bool pdl, int row0) {
     // Rows per CTA: one per sequence in decode; 2 or 3 when the batch averages that
     // many query tokens per sequence (multi-token verify), so that each sequence's
-    // keys are read once for all its rows; 4 for prefill-sized batches.
-    const int T = bv.total_q, B = bv.num_seqs;
+    // keys are read once for all its rows; 4 for prefill-sized batches.  The launch
+    // covers rows [row0, bv.total_q).
+    const int T = bv.total_q - row0, B = bv.num_seqs;
     const int G = T <= B ? 1 : T <= 2 * B ? 2 : T <= 3 * B ? 3 : 4;
     const int groups = (T + G - 1) / G;
     const int tiles_max = (bv.max_seq_len + kTileKeys - 1) / kTileKeys;
@@ -379,10 +381,10 @@ cudaError_t launch_indexer_fp8_tc(const void* q, const float* q_scale, const flo
     CUtensorMap tm_k, tm_q;
     cudaError_t e = make_map(&tm_k, k.data, (unsigned long long)k.num_pages * 64, 64);
     if (e != cudaSuccess) return e;
-    e = make_map(&tm_q, q, (unsigned long long)T * kHeads, G * kHeads);
+    e = make_map(&tm_q, q, (unsigned long long)bv.total_q * kHeads, G * kHeads);
     if (e != cudaSuccess) return e;
 
-    Params p{w, q_scale, k.scale, k.table, k.num_pages, k.bt_stride, bv, logits, ld, G, C, check};
+    Params p{w, q_scale, k.scale, k.table, k.num_pages, k.bt_stride, bv, logits, ld, G, C, row0, check};
     const size_t smem = 1024 + kStages * kTileBytes + (size_t)G * kRowBytes +
                         (size_t)G * kHeads * sizeof(float) + 16 * sizeof(uint64_t) + 16;
     dim3 grid(groups, chunks);

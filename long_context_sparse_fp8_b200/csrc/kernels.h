@@ -41,12 +41,12 @@ cudaError_t make_tensor_map_2d(CUtensorMap* m, const void* base, CUtensorMapData
 // Lightning Indexer on CUDA cores (fp32 q/k; any heads <= 64, dim <= 128, dim % 4 == 0).
 cudaError_t launch_indexer_generic(const void* q, const float* q_scale, const float* w, int heads,
                                    int dim, const CacheView& k, const BatchView& bv, float* logits,
-                                   long long ld, int* check, cudaStream_t st);
+                                   long long ld, int* check, cudaStream_t st, int row0 = 0);
 
 // Lightning Indexer on tcgen05 tensor cores (fp8 e4m3 q/k, 64 heads x 128 dims).
 cudaError_t launch_indexer_fp8_tc(const void* q, const float* q_scale, const float* w,
                                   const CacheView& k, const BatchView& bv, float* logits,
-                                  long long ld, int* check, cudaStream_t st, bool pdl = false);
+                                  long long ld, int* check, cudaStream_t st, bool pdl = false, int row0 = 0);
 
 // Writes n token rows of x (fp32 or bf16, [n][dim], dim % 16 == 0, dim <= 1024) into
 // cache rows slots[i] (negative: skipped) as fp8 e4m3 + amax/448 scale, bf16 or fp32.
@@ -54,9 +54,10 @@ cudaError_t launch_cache_store(const void* x, int x_dtype, int n, int dim, const
                                void* data, int cache_dtype, float* scale, long long num_rows,
                                int* check, cudaStream_t st);
 
-// Per-row top-k by radix select.
+// Per-row top-k by radix select.  Launches with row0 > 0 cover rows [row0, bv.total_q)
+// (the indexer writes, and the top-k reads, logits row t at (t - row0) * ld).
 cudaError_t launch_topk(const float* logits, long long ld, const BatchView& bv, int k, int* idx,
-                        int* check, cudaStream_t st, bool pdl = false);
+                        int* check, cudaStream_t st, bool pdl = false, int row0 = 0);
 
 // Sparse MLA on CUDA cores (fp32 q/KV).  nsplit > 1 writes partials (o/l, lse) to
 // o_part [T][nsplit][heads][d_v] / lse_part [T][nsplit][heads] instead of out/lse.

@@ -226,7 +226,7 @@ __device__ __forceinline__ void bitmap_to_list(Shared& sh, const uint32_t* bits,
 
 __global__ void __launch_bounds__(kThreads, 1)
 topk_kernel(const float* __restrict__ logits, long long ld, BatchView bv, int k,
-            int* __restrict__ idx, int* check, int words_cap, int stage_cap) {
+            int* __restrict__ idx, int* check, int words_cap, int stage_cap, int row0) {
     extern __shared__ __align__(16) uint8_t dyn[];
     int* hist = reinterpret_cast<int*>(dyn);                                   // [4][2048]
     uint32_t* ckey = reinterpret_cast<uint32_t*>(dyn + kCopies * 2048 * 4);      // [kCandCap]
@@ -236,7 +236,7 @@ topk_kernel(const float* __restrict__ logits, long long ld, BatchView bv, int k,
     uint32_t* skeys = eqmap + words_cap;                                         // [stage_cap]
     __shared__ Shared sh;
 
-    const int t = blockIdx.x, tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const int t = row0 + blockIdx.x, tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     pdl_trigger();
     int* out = idx + (long long)t * k;
     const RowInfo ri = row_info(bv, t, check);
@@ -249,7 +249,7 @@ topk_kernel(const float* __restrict__ logits, long long ld, BatchView bv, int k,
         for (int i = tid; i < k; i += kThreads) out[i] = i < n ? i : -1;
         return;
     }
-    const float* grow = logits + (long long)t * ld;
+    const float* grow = logits + (long long)(t - row0) * ld;
     const Row row{grow, skeys, stage_cap};
     const int words = (n + 31) >> 5;
     pdl_wait();                                  // the logits may come from the previous kernel
@@ -385,14 +385,14 @@ topk_kernel(const float* __restrict__ logits, long long ld, BatchView bv, int k,
 // the second writes).
 __global__ void __launch_bounds__(kThreads, 1)
 topk_long_kernel(const float* __restrict__ logits, long long ld, BatchView bv, int k,
-                 int* __restrict__ idx, int* check, int stage_cap) {
+                 int* __restrict__ idx, int* check, int stage_cap, int row0) {
     extern __shared__ __align__(16) uint8_t dyn[];
     int* hist = reinterpret_cast<int*>(dyn);                                // [4][2048]
     uint32_t* skeys = reinterpret_cast<uint32_t*>(dyn + kCopies * 2048 * 4);
     __shared__ Shared sh;
     __shared__ int s_gt[kWarps], s_eq[kWarps];
 
-    const int t = blockIdx.x, tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const int t = row0 + blockIdx.x, tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     int* out = idx + (long long)t * k;
     const RowInfo ri = row_info(bv, t, check);
     if (!ri.ok) {
@@ -404,7 +404,7 @@ topk_long_kernel(const float* __restrict__ logits, long long ld, BatchView bv, i
         for (int i = tid; i < k; i += kThreads) out[i] = i < n ? i : -1;
         return;
     }
-    const float* grow = logits + (long long)t * ld;
+    const float* grow = logits + (long long)(t - row0) * ld;
     const Row row{grow, skeys, stage_cap};
     pdl_wait();
     for (int i = tid; i < kCopies * 2048; i += kThreads) hist[i] = 0;
@@ -547,7 +547,7 @@ __device__ __forceinline__ void cluster_refine(Shared& sh, int* hist, ForEach fo
 
 __global__ void __launch_bounds__(kThreads, 1)
 topk_cluster_kernel(const float* __restrict__ logits, long long ld, BatchView bv, int k,
-                    int* __restrict__ idx, int* check, int words_cap, int stage_cap) {
+                    int* __restrict__ idx, int* check, int words_cap, int stage_cap, int row0) {
     extern __shared__ __align__(16) uint8_t dyn[];
     int* hist = reinterpret_cast<int*>(dyn);                                   // [4][2048]
     uint32_t* ckey = reinterpret_cast<uint32_t*>(dyn + kCopies * 2048 * 4);      // [kCCand]
@@ -561,7 +561,7 @@ topk_cluster_kernel(const float* __restrict__ logits, long long ld, BatchView bv
     uint32_t nrank_u;
     asm volatile("mov.u32 %0, %%cluster_nctarank;" : "=r"(nrank_u));
     const int nrank = (int)nrank_u, rank = (int)sm100::cluster_ctarank();
-    const int t = blockIdx.x / nrank, tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const int t = row0 + blockIdx.x / nrank, tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     pdl_trigger();
     int* out = idx + (long long)t * k;
     const RowInfo ri = row_info(bv, t, check);
@@ -579,7 +579,7 @@ topk_cluster_kernel(const float* __restrict__ logits, long long ld, BatchView bv
     // this CTA's segment of the row: [seg0, seg0 + sn), 32-aligned
     const int seg = (((n + nrank - 1) / nrank) + 31) & ~31;
     const int seg0 = min(n, rank * seg), sn = min(n, seg0 + seg) - seg0;
-    const float* grow = logits + (long long)t * ld + seg0;
+    const float* grow = logits + (long long)(t - row0) * ld + seg0;
     const Row row{grow, skeys, stage_cap};
     const int words = (sn + 31) >> 5;
     int use = 0;
@@ -716,14 +716,14 @@ topk_cluster_kernel(const float* __restrict__ logits, long long ld, BatchView bv
 }  // namespace
 
 cudaError_t launch_topk(const float* logits, long long ld, const BatchView& bv, int k, int* idx,
-                        int* check, cudaStream_t st, bool pdl) {
+                        int* check, cudaStream_t st, bool pdl, int row0) {
     const int hist_bytes = kCopies * 2048 * 4;
     const int words = ((bv.max_seq_len + 31) / 32 + 3) & ~3;
     // A few dozen long rows would leave most SMs idle with one CTA per row, and a row
     // beyond the staging capacity is re-read from L2: split each row over a cluster of
     // C CTAs instead.  (Rows of ~8K keys measured slower this way: the cluster barriers
     // and exchanges cost more than the split saves.)
-    const int T = bv.total_q;
+    const int T = bv.total_q - row0;
     const int C = T <= kNumSMs / 8 ? 8 : T <= kNumSMs / 4 ? 4 : T <= kNumSMs / 2 ? 2 : 1;
     const int cseg = (((bv.max_seq_len + C - 1) / C) + 31) & ~31;
     if (C > 1 && bv.max_seq_len >= 32768 && bv.max_seq_len > 2 * k && cseg <= 32 * kMaxWords) {
@@ -773,7 +773,7 @@ cudaError_t launch_topk(const float* logits, long long ld, const BatchView& bv, 
         if (clusters > 0) {
             cfg.numAttrs = pdl ? 2 : 1;
             e = cudaLaunchKernelEx(&cfg, topk_cluster_kernel, logits, ld, bv, k, idx, check, cwords,
-                                   stage);
+                                   stage, row0);
             if (e != cudaSuccess) return e;
             return cudaGetLastError();
         }
@@ -787,8 +787,8 @@ cudaError_t launch_topk(const float* logits, long long ld, const BatchView& bv, 
         cudaError_t e = cudaFuncSetAttribute(topk_kernel,
                                              cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
         if (e != cudaSuccess) return e;
-        e = launch_kernel(topk_kernel, dim3(bv.total_q), dim3(kThreads), smem, st, pdl, logits, ld,
-                          bv, k, idx, check, words, stage);
+        e = launch_kernel(topk_kernel, dim3(T), dim3(kThreads), smem, st, pdl, logits, ld,
+                          bv, k, idx, check, words, stage, row0);
         if (e != cudaSuccess) return e;
     } else {
         const int stage = (kSmemLimit - kStaticReserve - hist_bytes) / 4 & ~3;
@@ -796,8 +796,8 @@ cudaError_t launch_topk(const float* logits, long long ld, const BatchView& bv, 
         cudaError_t e = cudaFuncSetAttribute(topk_long_kernel,
                                              cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
         if (e != cudaSuccess) return e;
-        e = launch_kernel(topk_long_kernel, dim3(bv.total_q), dim3(kThreads), smem, st, pdl, logits,
-                          ld, bv, k, idx, check, stage);
+        e = launch_kernel(topk_long_kernel, dim3(T), dim3(kThreads), smem, st, pdl, logits,
+                          ld, bv, k, idx, check, stage, row0);
         if (e != cudaSuccess) return e;
     }
     return cudaGetLastError();

@@ -32,6 +32,7 @@ EXPORTED = (
     "dsa_sparse_mla_decode_workspace_size", "dsa_sparse_mla_decode",
     "dsa_sparse_mla_decode_noalloc",
     "dsa_cache_store",
+    "dsa_indexer_topk_workspace_size", "dsa_indexer_topk",
     "dsa_decode_workspace_size", "dsa_decode", "dsa_device_check", "dsa_last_error_message",
     "dsa_status_string", "dsa_version",
 )
@@ -88,6 +89,9 @@ def load_library(path: str = _LIB_PATH) -> ctypes.CDLL:
                         f32, CP, BP, P, P, ctypes.c_int, P, P, sz, P], ctypes.c_int),
         "dsa_cache_store": ([P, ctypes.c_int, i32, i32, P, P, ctypes.c_int, P, i64, P],
                             ctypes.c_int),
+        "dsa_indexer_topk_workspace_size": ([BP], sz),
+        "dsa_indexer_topk": ([P, ctypes.c_int, P, P, i32, i32, CP, BP, i32, P, P, sz, P],
+                             ctypes.c_int),
         "dsa_device_check": ([P, ctypes.POINTER(i32), i32], ctypes.c_int),
         "dsa_last_error_message": ([], ctypes.c_char_p),
         "dsa_status_string": ([ctypes.c_int], ctypes.c_char_p),
@@ -236,6 +240,28 @@ def dsa_decode(q_idx, q_idx_scale, w, k_cache: PagedCache, k: int, q, kv: PagedC
         float(softmax_scale), ctypes.byref(vc), ctypes.byref(bc), _ptr(idx_out), _ptr(out),
         dtype_code(out), _ptr(lse), _ptr(workspace), ws_bytes, _stream(stream)))
     return out
+
+
+def dsa_indexer_topk_workspace_size(batch: Batch) -> int:
+    bc = batch.c()
+    return int(load_library().dsa_indexer_topk_workspace_size(ctypes.byref(bc)))
+
+
+def dsa_indexer_topk(q, q_scale, w, k_cache: PagedCache, batch: Batch, k: int, idx,
+                     workspace=None, stream=None):
+    """Indexer + top-k over L2-sized blocks of query rows (no [T][L] logits); ``idx``
+    [T, k] int32 receives the same lists as dsa_indexer_logits + dsa_topk.  Without a
+    ``workspace`` (uint8, dsa_indexer_topk_workspace_size bytes) one is allocated."""
+    heads, dim = int(q.shape[-2]), int(q.shape[-1])
+    if workspace is None:
+        n = dsa_indexer_topk_workspace_size(batch)
+        workspace = torch.empty(max(n, 16), dtype=torch.uint8, device=q.device)
+    kc, bc = k_cache.c(), batch.c()
+    ws_bytes = workspace.numel() * workspace.element_size()
+    _check(load_library().dsa_indexer_topk(
+        _ptr(q), dtype_code(q), _ptr(q_scale), _ptr(w), heads, dim, ctypes.byref(kc),
+        ctypes.byref(bc), int(k), _ptr(idx), _ptr(workspace), ws_bytes, _stream(stream)))
+    return idx
 
 
 def dsa_cache_store(x, slot_mapping, cache_data, cache_scale=None, stream=None):

@@ -181,3 +181,19 @@ def test_cache_store_rejects_bad_arguments(case, expect):
 def test_cache_store_empty_is_a_no_op():
     assert L.load_library().dsa_cache_store(None, D.DSA_BF16, 0, 128, None, None,
                                             D.DSA_FP8_E4M3, None, 1, None) == D.DSA_OK
+
+
+def test_indexer_topk_checks_its_workspace():
+    lib = L.load_library()
+    b = _batch(1, 8192, 32768)
+    need = lib.dsa_indexer_topk_workspace_size(ctypes.byref(b))
+    assert need == 592 * 32768 * 4                 # a 74 MB block: 4 rows x 148 SMs
+    c = _cache()
+    st = lib.dsa_indexer_topk(FAKE, D.DSA_FP8_E4M3, None, FAKE, 64, 128, ctypes.byref(c),
+                              ctypes.byref(b), 2048, FAKE, FAKE2, need - 1, None)
+    assert st == D.DSA_ERR_WORKSPACE_TOO_SMALL, _status_msg()
+    st = lib.dsa_indexer_topk(FAKE, D.DSA_FP8_E4M3, None, FAKE, 64, 128, ctypes.byref(c),
+                              ctypes.byref(b), 2048, FAKE, None, need, None)
+    assert st == D.DSA_ERR_INVALID_ARGUMENT, _status_msg()
+    small = _batch(1, 8, 300)
+    assert lib.dsa_indexer_topk_workspace_size(ctypes.byref(small)) == 8 * 320 * 4

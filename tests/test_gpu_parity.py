@@ -235,6 +235,37 @@ def test_topk_cluster_split_matches_one_cta_per_row(kind):
     H.check_topk(full[sel], lg[sel], lg[sel], pos[sel], k)
 
 
+@pytest.mark.parametrize("which", ["prefill_32k", "fp32_blocks"])
+def test_indexer_topk_blocks_match_separate_calls(which):
+    """dsa_indexer_topk (L2-sized row blocks, no full logits matrix) selects exactly what
+    dsa_indexer_logits + dsa_topk select: 14 blocks of up to 592 rows on the 32K prefill
+    (FP8 tensor-core indexer), 2 blocks on an fp32 case (CUDA-core indexer)."""
+    if which == "prefill_32k":
+        wl = _wl("c3", W.prefill_32k)
+    else:
+        spec = W.Spec(name="blocks_f32", seq_lens=[40000, 30000], nq=[700, 300], topk=64,
+                      idx_heads=4, idx_dim=32, idx_fp8=False, w_std=0.5, heads=2, d_qk=80,
+                      d_v=64, mla_dtype="f32", softmax_scale=1.0 / math.sqrt(80.0), seed=31)
+        wl = W.make(spec, device="cuda")
+    s = wl.spec
+    batch, kc, _ = H.lib_args(wl)
+    logits = H.run_indexer(wl)
+    idx = H.run_topk(wl, logits)
+    ws_bytes = L.dsa_indexer_topk_workspace_size(batch)
+    ld = (s.max_seq_len + 63) // 64 * 64
+    assert ws_bytes < s.total_q * ld * 4 or s.total_q * ld * 4 <= 80 << 20
+    ws = torch.empty(ws_bytes, dtype=torch.uint8, device="cuda")
+    idx2 = torch.full_like(idx, -7)
+    L.dsa_indexer_topk(wl.q_idx, None, wl.w, kc, batch, s.topk, idx2, workspace=ws)
+    torch.cuda.synchronize()
+    assert L.dsa_device_check() == 0
+    assert torch.equal(idx, idx2)
+    rows = H.sample_rows(s.total_q, 6, seed=41)
+    pos = H.positions(wl)[rows]
+    g = logits.cpu().numpy()[rows]
+    H.check_topk(idx2.cpu().numpy()[rows], g, H.oracle_logits(wl, rows), pos, s.topk)
+
+
 def test_device_check_reports_bad_index_and_page():
     spec = W.Spec(name="chk", seq_lens=[300], nq=[4], topk=64, seed=5)
     wl = W.make(spec, device="cuda")
