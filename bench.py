@@ -61,6 +61,9 @@ def parse():
     p.add_argument("--workload", choices=sorted(WORKLOADS), default="decode_b32_ctx8192")
     p.add_argument("--no-cpu-baseline", action="store_true")
     p.add_argument("--cpu-seconds", type=float, default=12.0)
+    p.add_argument("--fp8-peak", action="store_true",
+                   help="measure the dense FP8 GEMM rate (torch._scaled_mm, e4m3, 8192^3, "
+                        "best of 10) and print it as one JSON line")
     return p.parse_args()
 
 
@@ -169,6 +172,38 @@ def measured_peaks():
         return d["hbm_gbs"], d["bf16_tflops"], "measured"
     except (OSError, KeyError, ValueError):
         return 6650.0, 1590.0, "fallback"
+
+
+def fp8_peak():
+    """The FP8 denominator: the measured figure recorded in profiles/fp8_peak.json (from
+    `bench.py --fp8-peak` on this pool), else 2x the measured bf16 peak (nominal ratio)."""
+    try:
+        with open(os.path.join(ROOT, "profiles", "fp8_peak.json")) as f:
+            return float(json.load(f)["fp8_tflops"]), "measured fp8 (torch._scaled_mm e4m3 8192^3)"
+    except (OSError, KeyError, ValueError):
+        return 2.0 * measured_peaks()[1], "2x measured bf16 (nominal ratio)"
+
+
+def measure_fp8_peak():
+    n = 8192
+    a = torch.randn(n, n, device="cuda").to(torch.float8_e4m3fn)
+    b = torch.randn(n, n, device="cuda").to(torch.float8_e4m3fn)
+    one = torch.ones((), device="cuda")
+    run = lambda: torch._scaled_mm(a, b.t(), scale_a=one, scale_b=one,  # noqa: E731
+                                   out_dtype=torch.bfloat16)
+    for _ in range(3):
+        run()
+    best = float("inf")
+    for _ in range(10):
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        run()
+        e1.record()
+        torch.cuda.synchronize()
+        best = min(best, e0.elapsed_time(e1))
+    return {"fp8_tflops": round(2 * n ** 3 / (best / 1e3) / 1e12, 1), "ms": round(best, 4),
+            "method": "torch._scaled_mm e4m3 x e4m3 -> bf16, 8192^3, best of 10 (CUDA events)",
+            "gpu": torch.cuda.get_device_name()}
 
 
 def ncu_traffic(workload: str, kernel_file: str):
@@ -332,13 +367,18 @@ def run_dsa(args, rank, world, dev):
         roof = {"bound": "hbm", "achieved": round(achieved, 1), "peak": hbm_gbs, "unit": "GB/s"}
     else:
         fl = work[dom]["flops"] / (mean_stage[dom] / 1e3) / 1e12
-        peak = bf16_tf * (2.0 if dom == "indexer" else 1.0)
+        peak = fp8_peak()[0] if dom == "indexer" else bf16_tf
         roof = {"bound": "tensor", "achieved": round(fl, 1), "peak": peak, "unit": "TFLOP/s"}
     roof["frac"] = round(roof["achieved"] / roof["peak"], 4)
     kernel_file = {"indexer": "indexer_tc.cu", "topk": "topk.cu", "mla": "mla_tc.cu"}[dom]
     roof["traffic"] = ncu_traffic(args.workload, kernel_file)
     roof["kernel"] = dom
-    roof["peak_source"] = f"{peak_kind} ({'burst' if roof['unit'] == 'GB/s' else 'burst bf16'})"
+    roof["peak_source"] = (f"{peak_kind} ({'burst' if roof['unit'] == 'GB/s' else 'burst bf16'})"
+                           if not (roof["unit"] == "TFLOP/s" and dom == "indexer") else fp8_peak()[1])
+    if mode == "prefill":
+        ix = work["indexer"]["flops"] / (mean_stage["indexer"] / 1e3) / 1e12
+        roof["indexer_fp8"] = {"achieved": round(ix, 1), "peak": fp8_peak()[0],
+                               "frac": round(ix / fp8_peak()[0], 4), "peak_source": fp8_peak()[1]}
     roof["stage_ms"] = {n: round(v, 4) for n, v in mean_stage.items()}
     roof["algorithmic_bytes_per_launch"] = work[dom]["bytes"]
     if mode == "prefill":
@@ -698,6 +738,9 @@ def _store_reference(args, world, dev):
 
 def main():
     args = parse()
+    if args.fp8_peak:
+        print(json.dumps(measure_fp8_peak()), flush=True)
+        return
     if args.impl == "reference":
         rank = int(os.environ.get("RANK", "0"))
         world = int(os.environ.get("WORLD_SIZE", "1"))
