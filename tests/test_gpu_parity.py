@@ -235,13 +235,17 @@ def test_topk_cluster_split_matches_one_cta_per_row(kind):
     H.check_topk(full[sel], lg[sel], lg[sel], pos[sel], k)
 
 
-@pytest.mark.parametrize("which", ["prefill_32k", "fp32_blocks"])
+@pytest.mark.parametrize("which", ["prefill_32k", "fp32_blocks", "ragged"])
 def test_indexer_topk_blocks_match_separate_calls(which):
     """dsa_indexer_topk (L2-sized row blocks, no full logits matrix) selects exactly what
     dsa_indexer_logits + dsa_topk select: 14 blocks of up to 592 rows on the 32K prefill
     (FP8 tensor-core indexer), 2 blocks on an fp32 case (CUDA-core indexer)."""
     if which == "prefill_32k":
         wl = _wl("c3", W.prefill_32k)
+    elif which == "ragged":
+        spec = W.Spec(name="ragged", seq_lens=[1, 63, 64, 65, 200, 2100, 3000, 2049],
+                      nq=[1, 5, 64, 2, 0, 7, 30, 3], topk=2048, seed=77)
+        wl = W.make(spec, device="cuda")
     else:
         spec = W.Spec(name="blocks_f32", seq_lens=[40000, 30000], nq=[700, 300], topk=64,
                       idx_heads=4, idx_dim=32, idx_fp8=False, w_std=0.5, heads=2, d_qk=80,
