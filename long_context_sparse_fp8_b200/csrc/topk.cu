@@ -26,10 +26,7 @@
 // than the bitmap capacity use a second kernel that refines over the whole row and
 // emits in two ordered sweeps.  Batches of a few dozen long rows (>= 32768 keys)
 // split every row over a thread-block cluster (topk_cluster_kernel, below).
-#include <algorithm>
-#include <mutex>
-#include <utility>
-#include <vector>
+#include <atomic>
 
 #include "kernels.h"
 #include "sm100.cuh"
@@ -750,25 +747,28 @@ cudaError_t launch_topk(const float* logits, long long ld, const BatchView& bv, 
         attr[1].val.programmaticStreamSerializationAllowed = 1;
         cfg.attrs = attr;
         cfg.numAttrs = 1;
-        // whether a cluster of this shape fits, asked once per (C, shared memory)
-        int clusters = 0;
-        {
-            static std::mutex mu;
-            static std::vector<std::pair<long long, int>> known;
-            const long long key = (long long)C << 32 | (long long)smem;
-            std::lock_guard<std::mutex> lk(mu);
-            auto it = std::find_if(known.begin(), known.end(),
-                                   [&](const std::pair<long long, int>& kv) { return kv.first == key; });
-            if (it != known.end()) {
-                clusters = it->second;
-            } else {
-                e = cudaOccupancyMaxActiveClusters(&clusters, topk_cluster_kernel, &cfg);
-                if (e != cudaSuccess) {
-                    (void)cudaGetLastError();
-                    clusters = 0;
-                }
-                known.emplace_back(key, clusters);
+        // whether a cluster of C CTAs fits, asked once per C at the largest shared-memory
+        // size this kernel uses (a smaller request then fits too)
+        static std::atomic<int> fits[4] = {{-1}, {-1}, {-1}, {-1}};   // C = 1, 2, 4, 8
+        const int slot = C == 2 ? 1 : C == 4 ? 2 : 3;
+        int clusters = fits[slot].load(std::memory_order_relaxed);
+        if (clusters < 0) {
+            const int max_smem = kSmemLimit - kStaticReserve;
+            cudaLaunchConfig_t probe = cfg;
+            probe.dynamicSmemBytes = max_smem;
+            int n = 0;
+            e = cudaFuncSetAttribute(topk_cluster_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                     max_smem);
+            if (e == cudaSuccess) e = cudaOccupancyMaxActiveClusters(&n, topk_cluster_kernel, &probe);
+            if (e != cudaSuccess) {
+                (void)cudaGetLastError();
+                n = 0;
             }
+            clusters = n > 0 ? 1 : 0;
+            fits[slot].store(clusters, std::memory_order_relaxed);
+            e = cudaFuncSetAttribute(topk_cluster_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                     (int)smem);
+            if (e != cudaSuccess) return e;
         }
         if (clusters > 0) {
             cfg.numAttrs = pdl ? 2 : 1;
