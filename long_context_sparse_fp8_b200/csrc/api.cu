@@ -205,7 +205,7 @@ dsa_status_t mla_check(const void* q, dsa_dtype_t q_dtype, int heads, int d_qk, 
 
 cudaError_t mla_launch(const MlaPlan& plan, const void* q, int heads, int d_qk, int d_v,
                        float scale, const BatchView& bv, const int* idx, int k, int nsplit,
-                       void* out, int out_dtype, float* lse, float* o_part, float* lse_part,
+                       void* out, int out_dtype, float* lse, void* o_part, float* lse_part,
                        int* check, cudaStream_t st, bool pdl = false) {
     // (pdl: the tensor-core kernel waits for its predecessor before reading idx; the
     // CUDA-core kernel does not, so it is always launched plainly)
@@ -213,7 +213,7 @@ cudaError_t mla_launch(const MlaPlan& plan, const void* q, int heads, int d_qk, 
         return launch_mla_tc(q, scale, plan.kv, bv, idx, k, nsplit, out, lse, o_part, lse_part,
                              check, st, pdl);
     return launch_mla_generic(q, heads, d_qk, d_v, scale, plan.kv, bv, idx, k, nsplit, out,
-                              out_dtype, lse, o_part, lse_part, check, st);
+                              out_dtype, lse, static_cast<float*>(o_part), lse_part, check, st);
 }
 
 // Split of each row's selection list for decode: enough CTAs to cover the GPU,
@@ -255,14 +255,16 @@ cudaError_t mla_decode_launch(const MlaPlan& plan, const void* q, int heads, int
     if (ns == 1)
         return mla_launch(plan, q, heads, d_qk, d_v, scale, bv, idx, k, 1, out, out_dtype, lse,
                           nullptr, nullptr, check, st, pdl);
-    float* o_part = static_cast<float*>(ws);
+    // partials o/l: fp16 from the tensor-core kernel (|o| <= max |v|, 11 significant
+    // bits), fp32 from the CUDA-core one; the workspace is sized for fp32 either way
+    void* o_part = ws;
     float* l_part = reinterpret_cast<float*>(
         static_cast<char*>(ws) + align_up((size_t)bv.total_q * ns * heads * d_v * 4, 256));
     cudaError_t e = mla_launch(plan, q, heads, d_qk, d_v, scale, bv, idx, k, ns, nullptr,
                                out_dtype, nullptr, o_part, l_part, check, st, pdl);
     if (e != cudaSuccess) return e;
-    return launch_mla_combine(o_part, l_part, bv.total_q, ns, heads, d_v, out, out_dtype, lse, st,
-                              pdl);
+    return launch_mla_combine(o_part, plan.kind == MlaKind::kTensorCore, l_part, bv.total_q, ns,
+                              heads, d_v, out, out_dtype, lse, st, pdl);
 }
 
 long long decode_ld(int max_seq_len) { return ((long long)max_seq_len + 63) / 64 * 64; }

@@ -68,7 +68,7 @@ cudaError_t launch_mla_generic(const void* q, int heads, int d_qk, int d_v, floa
 
 // Sparse MLA on tcgen05 tensor cores: bf16 q, bf16 or fp8 KV, 128 heads, 576 / 512.
 cudaError_t launch_mla_tc(const void* q, float scale, const CacheView& kv, const BatchView& bv,
-                          const int* idx, int k, int nsplit, void* out, float* lse, float* o_part,
+                          const int* idx, int k, int nsplit, void* out, float* lse, void* o_part,
                           float* lse_part, int* check, cudaStream_t st, bool pdl = false);
 
 // Size of the fixed device array behind dsa_sparse_mla_decode_noalloc
@@ -79,8 +79,8 @@ constexpr size_t kStaticScratchBytes = size_t(20) << 20;
 cudaError_t static_scratch(void** ptr);
 
 // Log-sum-exp merge of split partials into out (out_dtype) and lse.
-cudaError_t launch_mla_combine(const float* o_part, const float* lse_part, int total_q, int nsplit,
-                               int heads, int d_v, void* out, int out_dtype, float* lse,
-                               cudaStream_t st, bool pdl = false);
+cudaError_t launch_mla_combine(const void* o_part, bool half_part, const float* lse_part,
+                               int total_q, int nsplit, int heads, int d_v, void* out,
+                               int out_dtype, float* lse, cudaStream_t st, bool pdl = false);
 
 }  // namespace dsa

@@ -107,9 +107,21 @@ mla_generic_kernel(const void* __restrict__ q, int heads, int d_qk, int d_v, flo
 // With NS > 0 (= nsplit, known at compile time) every partial a thread needs is
 // loaded before any is used, so the loads overlap instead of forming a dependent
 // chain; NS = 0 handles any nsplit <= 16 the same way in a fixed-size frame.
-template <int NS>
+template <typename PT>
+__device__ __forceinline__ float4 load_part4(const PT* p) {
+    if constexpr (sizeof(PT) == 4) {
+        return __ldg(reinterpret_cast<const float4*>(p));
+    } else {
+        const uint2 u = __ldg(reinterpret_cast<const uint2*>(p));
+        const float2 a = __half22float2(*reinterpret_cast<const __half2*>(&u.x));
+        const float2 b = __half22float2(*reinterpret_cast<const __half2*>(&u.y));
+        return make_float4(a.x, a.y, b.x, b.y);
+    }
+}
+
+template <int NS, typename PT>
 __global__ void __launch_bounds__(256)
-mla_combine_kernel(const float* __restrict__ o_part, const float* __restrict__ lse_part,
+mla_combine_kernel(const PT* __restrict__ o_part, const float* __restrict__ lse_part,
                    int nsplit_rt, int heads, int d_v, void* __restrict__ out, int out_dtype,
                    float* __restrict__ lse) {
     constexpr int kMaxSplit = NS > 0 ? NS : 16;
@@ -127,7 +139,7 @@ mla_combine_kernel(const float* __restrict__ o_part, const float* __restrict__ l
         if (i < nsplit) {
             const long long pb = ((long long)t * nsplit + i) * heads + h;
             li[i] = __ldg(lse_part + pb);
-            ov[i] = __ldg(reinterpret_cast<const float4*>(o_part + pb * d_v) + d4);
+            ov[i] = load_part4(o_part + pb * d_v + 4 * d4);
         }
     }
     float mx = -INFINITY;
@@ -175,21 +187,37 @@ cudaError_t launch_mla_generic(const void* q, int heads, int d_qk, int d_v, floa
     return cudaGetLastError();
 }
 
-cudaError_t launch_mla_combine(const float* o_part, const float* lse_part, int total_q, int nsplit,
-                               int heads, int d_v, void* out, int out_dtype, float* lse,
-                               cudaStream_t st, bool pdl) {
+namespace {
+
+template <typename PT>
+cudaError_t combine_for(const PT* o_part, const float* lse_part, int total_q, int nsplit,
+                        int heads, int d_v, void* out, int out_dtype, float* lse, cudaStream_t st,
+                        bool pdl) {
     // d_v % 4 == 0 and d_v <= 512 (validated by the callers)
     const int per_head = d_v / 4;
     const int heads_per_block = per_head >= 256 ? 1 : 256 / per_head;
     dim3 grid(total_q, (heads + heads_per_block - 1) / heads_per_block);
     const int threads = per_head * heads_per_block;
-    auto kern = nsplit == 2 ? mla_combine_kernel<2> : nsplit == 3 ? mla_combine_kernel<3>
-              : nsplit == 4 ? mla_combine_kernel<4> : nsplit == 8 ? mla_combine_kernel<8>
-                                                                  : mla_combine_kernel<0>;
+    auto kern = nsplit == 2 ? mla_combine_kernel<2, PT> : nsplit == 3 ? mla_combine_kernel<3, PT>
+              : nsplit == 4 ? mla_combine_kernel<4, PT> : nsplit == 8 ? mla_combine_kernel<8, PT>
+                                                                      : mla_combine_kernel<0, PT>;
     cudaError_t e = launch_kernel(kern, grid, dim3(threads), 0, st, pdl, o_part, lse_part, nsplit,
                                   heads, d_v, out, out_dtype, lse);
     if (e != cudaSuccess) return e;
     return cudaGetLastError();
+}
+
+}  // namespace
+
+// Partials: fp16 from the tensor-core kernel, fp32 from the CUDA-core one.
+cudaError_t launch_mla_combine(const void* o_part, bool half_part, const float* lse_part,
+                               int total_q, int nsplit, int heads, int d_v, void* out,
+                               int out_dtype, float* lse, cudaStream_t st, bool pdl) {
+    return half_part
+               ? combine_for(static_cast<const __half*>(o_part), lse_part, total_q, nsplit, heads,
+                             d_v, out, out_dtype, lse, st, pdl)
+               : combine_for(static_cast<const float*>(o_part), lse_part, total_q, nsplit, heads,
+                             d_v, out, out_dtype, lse, st, pdl);
 }
 
 }  // namespace dsa

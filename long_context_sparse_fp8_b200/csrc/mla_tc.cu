@@ -91,7 +91,7 @@ struct Params {
     float sc_log2;             // softmax_scale * log2(e)
     __nv_bfloat16* out;
     float* lse;
-    float* o_part;
+    __half* o_part;            // split partials o / l in fp16 (|o| <= max |v|)
     float* lse_part;
     int* check;
 };
@@ -556,7 +556,7 @@ mla_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const Params p) {
             if (vh == 0 && p.lse) p.lse[(long long)t * kHeads + h] = lse_v;
         } else {
             const long long pb = ((long long)t * p.nsplit + split) * kHeads + h;
-            float4* orow = reinterpret_cast<float4*>(p.o_part + pb * 512 + vh * 256);
+            uint4* orow = reinterpret_cast<uint4*>(p.o_part + pb * 512 + vh * 256);
 #pragma unroll 1
             for (int cc = 0; cc < 8; ++cc) {
                 uint32_t o[32];
@@ -565,12 +565,16 @@ mla_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const Params p) {
                     tmem_ld_wait();
                 }
 #pragma unroll
-                for (int q4 = 0; q4 < 8; ++q4)
-                    orow[cc * 8 + q4] = have ? make_float4(__uint_as_float(o[4 * q4]) * inv,
-                                                           __uint_as_float(o[4 * q4 + 1]) * inv,
-                                                           __uint_as_float(o[4 * q4 + 2]) * inv,
-                                                           __uint_as_float(o[4 * q4 + 3]) * inv)
-                                             : make_float4(0.f, 0.f, 0.f, 0.f);
+                for (int q8 = 0; q8 < 4; ++q8) {
+                    uint4 w = make_uint4(0u, 0u, 0u, 0u);
+                    if (have) {
+                        w.x = pack_f16(__uint_as_float(o[8 * q8 + 0]) * inv, __uint_as_float(o[8 * q8 + 1]) * inv);
+                        w.y = pack_f16(__uint_as_float(o[8 * q8 + 2]) * inv, __uint_as_float(o[8 * q8 + 3]) * inv);
+                        w.z = pack_f16(__uint_as_float(o[8 * q8 + 4]) * inv, __uint_as_float(o[8 * q8 + 5]) * inv);
+                        w.w = pack_f16(__uint_as_float(o[8 * q8 + 6]) * inv, __uint_as_float(o[8 * q8 + 7]) * inv);
+                    }
+                    orow[cc * 4 + q8] = w;
+                }
             }
             if (vh == 0) p.lse_part[pb] = lse_v;
         }
@@ -585,7 +589,7 @@ mla_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const Params p) {
 }  // namespace
 
 cudaError_t launch_mla_tc(const void* q, float scale, const CacheView& kv, const BatchView& bv,
-                          const int* idx, int k, int nsplit, void* out, float* lse, float* o_part,
+                          const int* idx, int k, int nsplit, void* out, float* lse, void* o_part,
                           float* lse_part, int* check, cudaStream_t st, bool pdl) {
     Params p;
     p.q = reinterpret_cast<const uint4*>(q);
@@ -602,7 +606,7 @@ cudaError_t launch_mla_tc(const void* q, float scale, const CacheView& kv, const
     p.sc_log2 = scale * 1.4426950408889634f;
     p.out = reinterpret_cast<__nv_bfloat16*>(out);
     p.lse = lse;
-    p.o_part = o_part;
+    p.o_part = static_cast<__half*>(o_part);
     p.lse_part = lse_part;
     p.check = check;
     CUtensorMap tm_q;
