@@ -21,7 +21,7 @@ indexer_generic_kernel(const void* __restrict__ q, const float* __restrict__ q_s
                        float* __restrict__ logits, long long ld, int row0, int* check) {
     extern __shared__ float sm[];
     const int t = row0 + blockIdx.x, tile = blockIdx.y, tid = threadIdx.x;
-    logits -= (long long)row0 * ld;          // row t of the launch is logits row t - row0
+    float* lrow = logits + (long long)blockIdx.x * ld;   // row t is logits row t - row0
     const RowInfo ri = row_info(bv, t, check);
     if (!ri.ok) return;
     const int s0 = tile * kIndexerPage;
@@ -45,7 +45,7 @@ indexer_generic_kernel(const void* __restrict__ q, const float* __restrict__ q_s
     const long long r0 = page_row0;
     if (r0 < 0) {  // bad page: recorded; the tile's scores are -inf
         for (int i = tid; i < kIndexerPage; i += kThreads)
-            if (s0 + i <= ri.pos) logits[(long long)t * ld + s0 + i] = -INFINITY;
+            if (s0 + i <= ri.pos) lrow[s0 + i] = -INFINITY;
         return;
     }
     for (int i = tid; i < kIndexerPage * dim; i += kThreads)
@@ -68,8 +68,8 @@ indexer_generic_kernel(const void* __restrict__ q, const float* __restrict__ q_s
     if (part == 0) {
         const int s = s0 + key;
         const float qsc = q_scale ? __ldg(q_scale + t) : 1.0f;
-        if (s <= ri.pos) logits[(long long)t * ld + s] = kscale[key] * qsc * acc;
-        else if (s < ld) logits[(long long)t * ld + s] = -INFINITY;
+        if (s <= ri.pos) lrow[s] = kscale[key] * qsc * acc;
+        else if (s < ld) lrow[s] = -INFINITY;
     }
 }
 
