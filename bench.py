@@ -48,6 +48,7 @@ WORKLOADS = {
     "prefill_L32768_q8192": (W.prefill_32k, "prefill"),
     "decode_b64_ctx64k-128k_fp8kv": (W.decode_b64_128k, "decode"),
     "decode_mtp2_b32_ctx8192": (W.decode_mtp_b32_8k, "decode"),
+    "prefill_L131072_chunk15": (lambda: W.chunked_prefill_128k(15), "prefill"),
     "store_L131072_fp8": (W.store_prompt_128k, "store"),
 }
 

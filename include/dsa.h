@@ -234,7 +234,7 @@ DSA_API dsa_status_t dsa_decode(const void* q_idx, dsa_dtype_t q_idx_dtype,
  * dsa_indexer_topk -- the indexer and the top-k without the full logits matrix
  * ("SGLang Day-0 support for DeepSeek-V3.2", its launch lines' FUSE_TOPK switch: the
  * selection fused with the scoring).  The query rows are processed in blocks whose
- * logits take at most 80 MB of the L2 (592 rows at 32K context, 160 at 128K); each
+ * logits take at most 80 MB of the L2 (592 rows at 32K context, 148 at 128K); each
  * block's logits go to the workspace and are selected from at once, so they do not
  * round-trip through HBM and the memory needed is one block, not [T][L].
  * Arguments and results are those of dsa_indexer_logits followed by dsa_topk

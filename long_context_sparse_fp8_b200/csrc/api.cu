@@ -466,15 +466,20 @@ DSA_API dsa_status_t dsa_decode(const void* q_idx, dsa_dtype_t q_idx_dtype,
 }
 
 // Rows per block of dsa_indexer_topk: the logits of one block take at most 80 MB of the
-// 126 MB L2, so the top-k reads them while they are still on chip; where that allows
-// several hundred rows, a multiple of 592 (4 rows per indexer CTA x 148 SMs, and one
-// top-k CTA per row) so that both kernels run whole waves.
+// 126 MB L2, so the top-k reads them while they are still on chip.  Where that allows
+// 148 rows or more, 148 x 2^m rows: the top-k runs one CTA per row and the indexer 4 rows
+// per CTA over 592 / (rows / 4) key chunks, so both fill whole waves of the 148 SMs.
 constexpr size_t kL2BlockBytes = (size_t)80 << 20;
-constexpr int kWaveRows = 4 * kNumSMs;
 
 int indexer_topk_block_rows(int total_q, long long ld) {
-    long long rows = (long long)(kL2BlockBytes / ((size_t)ld * sizeof(float)));
-    rows = rows >= kWaveRows ? rows / kWaveRows * kWaveRows : rows & ~3LL;
+    const long long budget = (long long)(kL2BlockBytes / ((size_t)ld * sizeof(float)));
+    long long rows;
+    if (budget >= kNumSMs) {
+        rows = kNumSMs;
+        while (rows * 2 <= budget) rows *= 2;
+    } else {
+        rows = budget & ~3LL;
+    }
     if (rows < 4) rows = 4;
     if (rows > total_q) rows = total_q;
     return (int)rows;

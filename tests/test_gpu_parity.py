@@ -239,7 +239,7 @@ def test_topk_cluster_split_matches_one_cta_per_row(kind):
 def test_indexer_topk_blocks_match_separate_calls(which):
     """dsa_indexer_topk (L2-sized row blocks, no full logits matrix) selects exactly what
     dsa_indexer_logits + dsa_topk select: 14 blocks of up to 592 rows on the 32K prefill
-    (FP8 tensor-core indexer), 2 blocks on an fp32 case (CUDA-core indexer)."""
+    (FP8 tensor-core indexer), 4 blocks on an fp32 case (CUDA-core indexer)."""
     if which == "prefill_32k":
         wl = _wl("c3", W.prefill_32k)
     elif which == "ragged":
