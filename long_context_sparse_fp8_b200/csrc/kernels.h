@@ -67,6 +67,8 @@ cudaError_t launch_mla_generic(const void* q, int heads, int d_qk, int d_v, floa
                                float* lse_part, int* check, cudaStream_t st);
 
 // Sparse MLA on tcgen05 tensor cores: bf16 q, bf16 or fp8 KV, 128 heads, 576 / 512.
+// nsplit > 1 writes partials o/l in fp16 to o_part [T][nsplit][128][512] (each is
+// bounded by the largest V value) and lse to lse_part [T][nsplit][128] fp32.
 cudaError_t launch_mla_tc(const void* q, float scale, const CacheView& kv, const BatchView& bv,
                           const int* idx, int k, int nsplit, void* out, float* lse, void* o_part,
                           float* lse_part, int* check, cudaStream_t st, bool pdl = false);
@@ -78,7 +80,8 @@ constexpr size_t kStaticScratchBytes = size_t(20) << 20;
 // Address of that array on the current device (looked up once per device).
 cudaError_t static_scratch(void** ptr);
 
-// Log-sum-exp merge of split partials into out (out_dtype) and lse.
+// Log-sum-exp merge of split partials (fp16 when half_part, else fp32) into out
+// (out_dtype) and lse.
 cudaError_t launch_mla_combine(const void* o_part, bool half_part, const float* lse_part,
                                int total_q, int nsplit, int heads, int d_v, void* out,
                                int out_dtype, float* lse, cudaStream_t st, bool pdl = false);
