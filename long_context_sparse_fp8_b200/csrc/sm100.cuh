@@ -87,30 +87,6 @@ __device__ __forceinline__ bool mbar_wait_warp(uint64_t* bar, uint32_t parity, i
     return ok;
 }
 
-// Same wait with cluster-scope acquire: for data a peer CTA wrote into this
-// CTA's shared memory before arriving remotely.
-__device__ __forceinline__ bool mbar_try_wait_cluster(uint64_t* bar, uint32_t parity) {
-    uint32_t ok;
-    asm volatile(
-        "{\n\t.reg .pred p;\n\t"
-        "mbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2;\n\t"
-        "selp.u32 %0, 1, 0, p;\n\t}"
-        : "=r"(ok) : "r"(smem_u32(bar)), "r"(parity) : "memory");
-    return ok != 0;
-}
-
-__device__ __forceinline__ bool mbar_wait_cluster(uint64_t* bar, uint32_t parity, int* check) {
-    if (mbar_try_wait_cluster(bar, parity)) return true;
-    const long long t0 = clock64();
-    while (!mbar_try_wait_cluster(bar, parity)) {
-        if (clock64() - t0 > kWaitLimitCycles) {
-            report(check, kCheckTimeout);
-            return false;
-        }
-    }
-    return true;
-}
-
 // ---------------------------------------------------------------- clusters
 __device__ __forceinline__ uint32_t cluster_ctarank() {
     uint32_t r;
@@ -125,32 +101,8 @@ __device__ __forceinline__ uint32_t mapa(uint32_t saddr, uint32_t rank) {
     return r;
 }
 
-__device__ __forceinline__ void st_cluster_v4(uint32_t caddr, float a, float b, float c, float d) {
-    asm volatile("st.shared::cluster.v4.f32 [%0], {%1, %2, %3, %4};"
-                 ::"r"(caddr), "f"(a), "f"(b), "f"(c), "f"(d) : "memory");
-}
-
-// Arrive on a peer CTA's mbarrier, releasing this thread's prior writes cluster-wide.
-__device__ __forceinline__ void mbar_arrive_remote(uint32_t caddr) {
-    asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];"
-                 ::"r"(caddr) : "memory");
-}
-
-// Asynchronous 16-byte store into a peer CTA's shared memory that completes its
-// bytes on the peer's mbarrier (no fence needed on either side).
-__device__ __forceinline__ void st_async_v4(uint32_t caddr, float a, float b, float c, float d,
-                                            uint32_t cbar) {
-    asm volatile(
-        "st.async.shared::cluster.mbarrier::complete_tx::bytes.v4.f32 [%0], {%1, %2, %3, %4}, [%5];"
-        ::"r"(caddr), "f"(a), "f"(b), "f"(c), "f"(d), "r"(cbar) : "memory");
-}
-
-// Plain arrive on a peer CTA's mbarrier (signals a consumed buffer; no data).
-__device__ __forceinline__ void mbar_arrive_peer(uint32_t caddr) {
-    asm volatile("mbarrier.arrive.shared::cluster.b64 _, [%0];" ::"r"(caddr) : "memory");
-}
-
-// All threads of both CTAs (must be executed convergently by every warp).
+// Barrier over every thread of every CTA of the cluster (executed convergently by
+// every warp).
 __device__ __forceinline__ void cluster_sync() {
     asm volatile("barrier.cluster.arrive.release.aligned;\n\t"
                  "barrier.cluster.wait.acquire.aligned;" ::: "memory");
