@@ -269,8 +269,10 @@ DSA_API dsa_status_t dsa_indexer_topk(const void* q, dsa_dtype_t q_dtype, const 
  *   cache_scale   [num_rows] fp32, written for an FP8 cache; ignored (may be
  *                 NULL) for BF16 / F32 caches
  * FP8 cache: scale = amax / 448 in fp32 with amax = max |x_e| of the row (1 for
- * an all-zero row), code_e = e4m3(x_e / scale): the quotient is an IEEE fp32
- * division, rounded to e4m3 to nearest even and saturated at +-448.  BF16
+ * an all-zero row, or when amax / 448 underflows to 0), code_e = e4m3(x_e /
+ * scale): the quotient is an IEEE fp32 division (correctly rounded), rounded to
+ * e4m3 to nearest even and saturated at +-448, so that code * scale
+ * dequantises.  BF16
  * cache: x rounded to nearest even.  F32 cache: x widened exactly.
  * dim must be a multiple of 16 in [16, 1024]; pointers 16-byte aligned
  * (slot_mapping 8, cache_scale 4).  A slot >= num_rows is skipped and recorded

@@ -12,10 +12,19 @@
 // Rows are spread over lane groups: 16 lanes per row when the row has at most 16
 // chunks of 8 elements (the 128-wide indexer key), else 32.  Each lane group takes four
 // rows per pass, so every warp keeps 4-8 rows of loads in flight (up to four 16-B or
-// 32-B loads per lane per row, all issued before use, kept packed until converted); |x| is max-reduced within the
-// group, the factor 448/amax is formed once per row, and each lane converts and
-// stores its chunks (8 B of e4m3 codes, 16 B of bf16 or 32 B of fp32).  HBM-bound:
-// dim x (input + output bytes) + 4 B scale + 8 B slot per token.
+// 32-B loads per lane per row, all issued before use, kept packed until converted);
+// |x| is max-reduced within the group, the scale amax/448 is formed once per row, and
+// each lane converts and stores its chunks (8 B of e4m3 codes, 16 B of bf16 or 32 B of
+// fp32).  HBM-bound: dim x (input + output bytes) + 4 B scale + 8 B slot per token.
+//
+// The FP8 codes are e4m3(x / scale) with the quotient correctly rounded to fp32.  A
+// division per element would make the kernel compute-bound, so each quotient is first
+// taken as x * (1/scale), which lies within 3 fp32 ulps of the correctly rounded
+// quotient; when the e4m3 codes of that product scaled by (1 - 2^-20) and by
+// (1 + 2^-20) agree, every value in between -- the exact quotient among them -- has the
+// same code (rounding is monotone), and otherwise (a product next to an e4m3 rounding
+// boundary, about one element in 10^5) the code is taken from the division itself.
+// Scales below the smallest normal fp32, whose reciprocal may overflow, divide always.
 #include <atomic>
 
 #include "common.cuh"
@@ -62,6 +71,21 @@ __device__ __forceinline__ uint32_t e4m3x2(float lo, float hi) {
     uint16_t r;
     asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(r) : "f"(hi), "f"(lo));
     return r;
+}
+
+// e4m3 codes of a / sc and b / sc, the quotients correctly rounded to fp32 (see the
+// head of the file); rcp = 1/sc correctly rounded.
+__device__ __forceinline__ uint32_t e4m3x2_div(float a, float b, float sc, float rcp,
+                                               bool divide_all) {
+    if (!divide_all) {
+        const float qa = __fmul_rn(a, rcp), qb = __fmul_rn(b, rcp);
+        const uint32_t code = e4m3x2(qa, qb);
+        const float dn = 1.0f - 0x1p-20f, up = 1.0f + 0x1p-20f;
+        const uint32_t lo = e4m3x2(__fmul_rn(qa, dn), __fmul_rn(qb, dn));
+        const uint32_t hi = e4m3x2(__fmul_rn(qa, up), __fmul_rn(qb, up));
+        if (lo == code && hi == code) return code;
+    }
+    return e4m3x2(__fdiv_rn(a, sc), __fdiv_rn(b, sc));
 }
 
 __device__ __forceinline__ uint32_t bf16x2(float lo, float hi) {
@@ -116,9 +140,12 @@ __global__ void __launch_bounds__(kThreads) cache_store_kernel(
                 for (int o = LPR / 2; o > 0; o >>= 1)
                     amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
                 if (slot[u] < 0) continue;
-                // codes = e4m3(x * 448/amax); the factor is capped at the largest finite
-                // fp32 (amax = 0 then gives zero codes)
-                const float inv = fminf(__fdiv_rn(448.0f, amax), 3.40282347e38f);
+                // scale = amax / 448 (1 for a zero row or an underflowed quotient);
+                // codes = e4m3(x / scale)
+                float sc = __fdiv_rn(amax, 448.0f);
+                if (!(sc > 0.f)) sc = 1.0f;
+                const float rcp = __frcp_rn(sc);
+                const bool divide_all = sc < 1.17549435e-38f;     // subnormal scale
                 uint8_t* dst = static_cast<uint8_t*>(data) + slot[u] * dim;
 #pragma unroll
                 for (int r = 0; r < CPL; ++r) {
@@ -127,11 +154,11 @@ __global__ void __launch_bounds__(kThreads) cache_store_kernel(
                     uint32_t q[4];
 #pragma unroll
                     for (int e = 0; e < 4; ++e)
-                        q[e] = e4m3x2(__fmul_rn(elem<XT>(v[u][r], 2 * e), inv),
-                                      __fmul_rn(elem<XT>(v[u][r], 2 * e + 1), inv));
+                        q[e] = e4m3x2_div(elem<XT>(v[u][r], 2 * e), elem<XT>(v[u][r], 2 * e + 1), sc,
+                                          rcp, divide_all);
                     *reinterpret_cast<uint2*>(dst + 8 * c) = make_uint2(q[0] | (q[1] << 16), q[2] | (q[3] << 16));
                 }
-                if (gl == 0) scale[slot[u]] = amax > 0.f ? __fdiv_rn(amax, 448.0f) : 1.0f;
+                if (gl == 0) scale[slot[u]] = sc;
             } else if constexpr (CT == kBF16) {
                 if (slot[u] < 0) continue;
                 uint16_t* dst = static_cast<uint16_t*>(data) + slot[u] * dim;

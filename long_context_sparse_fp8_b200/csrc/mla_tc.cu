@@ -527,7 +527,9 @@ mla_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const Params p) {
             tc_fence_before();
             mbar_arrive(&pfull[j & 1]);
         }
-        // ---- epilogue: O_v / l and lse
+        // ---- epilogue: O_v / l and lse (after the predecessor kernel: an earlier kernel
+        // of the stream may still read the output or partial buffers)
+        pdl_wait();
         const bool have = alive && n_tiles > 0 &&
                           mbar_wait_warp(&pvdone[(n_tiles - 1) & 1], ((n_tiles - 1) >> 1) & 1, p.check);
         tc_fence_after();

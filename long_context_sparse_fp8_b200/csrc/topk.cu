@@ -26,7 +26,7 @@
 // than the bitmap capacity use a second kernel that refines over the whole row and
 // emits in two ordered sweeps.  Batches of a few dozen long rows (>= 32768 keys)
 // split every row over a thread-block cluster (topk_cluster_kernel, below).
-#include <atomic>
+#include <mutex>
 
 #include "kernels.h"
 #include "sm100.cuh"
@@ -237,6 +237,9 @@ topk_kernel(const float* __restrict__ logits, long long ld, BatchView bv, int k,
     pdl_trigger();
     int* out = idx + (long long)t * k;
     const RowInfo ri = row_info(bv, t, check);
+    // the logits may come from the previous kernel, and an earlier kernel of the stream
+    // may still read the selection buffer: wait before the first load or store
+    pdl_wait();
     if (!ri.ok) {
         for (int i = tid; i < k; i += kThreads) out[i] = -1;
         return;
@@ -249,7 +252,6 @@ topk_kernel(const float* __restrict__ logits, long long ld, BatchView bv, int k,
     const float* grow = logits + (long long)(t - row0) * ld;
     const Row row{grow, skeys, stage_cap};
     const int words = (n + 31) >> 5;
-    pdl_wait();                                  // the logits may come from the previous kernel
 
     // ---- 1. stage + top-bit histogram ------------------------------------------
     for (int i = tid; i < kCopies * 2048; i += kThreads) hist[i] = 0;
@@ -392,6 +394,7 @@ topk_long_kernel(const float* __restrict__ logits, long long ld, BatchView bv, i
     const int t = row0 + blockIdx.x, tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     int* out = idx + (long long)t * k;
     const RowInfo ri = row_info(bv, t, check);
+    pdl_wait();                                  // before the first load or store (see topk_kernel)
     if (!ri.ok) {
         for (int i = tid; i < k; i += kThreads) out[i] = -1;
         return;
@@ -403,7 +406,6 @@ topk_long_kernel(const float* __restrict__ logits, long long ld, BatchView bv, i
     }
     const float* grow = logits + (long long)(t - row0) * ld;
     const Row row{grow, skeys, stage_cap};
-    pdl_wait();
     for (int i = tid; i < kCopies * 2048; i += kThreads) hist[i] = 0;
     __syncthreads();
     stage_and_histogram(grow, n, skeys, stage_cap, hist);
@@ -562,6 +564,7 @@ topk_cluster_kernel(const float* __restrict__ logits, long long ld, BatchView bv
     pdl_trigger();
     int* out = idx + (long long)t * k;
     const RowInfo ri = row_info(bv, t, check);
+    pdl_wait();                                  // before the first load or store (see topk_kernel)
     if (!ri.ok) {
         if (rank == 0)
             for (int i = tid; i < k; i += kThreads) out[i] = -1;
@@ -580,7 +583,6 @@ topk_cluster_kernel(const float* __restrict__ logits, long long ld, BatchView bv
     const Row row{grow, skeys, stage_cap};
     const int words = (sn + 31) >> 5;
     int use = 0;
-    pdl_wait();
 
     // ---- 1. stage + top-bit histogram, summed over the cluster ---------------------
     for (int i = tid; i < kCopies * 2048; i += kThreads) hist[i] = 0;
@@ -710,10 +712,68 @@ topk_cluster_kernel(const float* __restrict__ logits, long long ld, BatchView bv
     }
 }
 
+
+// Per-device launch state: every top-k kernel's dynamic shared-memory limit is raised
+// once to the largest size any launch asks for (so no launch ever lowers it under a
+// launch on another host thread), and whether a cluster of 2, 4 or 8 CTAs at that
+// size fits on the device is asked once.
+constexpr int kMaxDynSmem = kSmemLimit - kStaticReserve;
+constexpr int kMaxDevices = 64;
+
+struct TopkDeviceState {
+    std::once_flag once;
+    cudaError_t err = cudaSuccess;
+    bool cluster_fits[4] = {false, false, false, false};   // index: C = 1, 2, 4, 8
+};
+TopkDeviceState g_topk_dev[kMaxDevices];
+
+cudaError_t topk_device_state(const TopkDeviceState** out) {
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
+    TopkDeviceState& s = g_topk_dev[dev];
+    std::call_once(s.once, [&s] {
+        for (auto kern : {topk_kernel, topk_cluster_kernel}) {
+            s.err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, kMaxDynSmem);
+            if (s.err != cudaSuccess) return;
+        }
+        s.err = cudaFuncSetAttribute(topk_long_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                     kMaxDynSmem);
+        if (s.err != cudaSuccess) return;
+        for (int slot = 1; slot < 4; ++slot) {
+            cudaLaunchConfig_t probe = {};
+            const unsigned C = 1u << slot;
+            probe.gridDim = dim3(C);
+            probe.blockDim = dim3(kThreads);
+            probe.dynamicSmemBytes = kMaxDynSmem;
+            cudaLaunchAttribute attr[1];
+            attr[0].id = cudaLaunchAttributeClusterDimension;
+            attr[0].val.clusterDim.x = C;
+            attr[0].val.clusterDim.y = 1;
+            attr[0].val.clusterDim.z = 1;
+            probe.attrs = attr;
+            probe.numAttrs = 1;
+            int n = 0;
+            if (cudaOccupancyMaxActiveClusters(&n, topk_cluster_kernel, &probe) != cudaSuccess) {
+                (void)cudaGetLastError();
+                n = 0;
+            }
+            s.cluster_fits[slot] = n > 0;
+        }
+    });
+    if (s.err != cudaSuccess) return s.err;
+    *out = &s;
+    return cudaSuccess;
+}
+
 }  // namespace
 
 cudaError_t launch_topk(const float* logits, long long ld, const BatchView& bv, int k, int* idx,
                         int* check, cudaStream_t st, bool pdl, int row0) {
+    const TopkDeviceState* ds = nullptr;
+    cudaError_t de = topk_device_state(&ds);
+    if (de != cudaSuccess) return de;
     const int hist_bytes = kCopies * 2048 * 4;
     const int words = ((bv.max_seq_len + 31) / 32 + 3) & ~3;
     // A few dozen long rows would leave most SMs idle with one CTA per row, and a row
@@ -723,16 +783,15 @@ cudaError_t launch_topk(const float* logits, long long ld, const BatchView& bv, 
     const int T = bv.total_q - row0;
     const int C = T <= kNumSMs / 8 ? 8 : T <= kNumSMs / 4 ? 4 : T <= kNumSMs / 2 ? 2 : 1;
     const int cseg = (((bv.max_seq_len + C - 1) / C) + 31) & ~31;
-    if (C > 1 && bv.max_seq_len >= 32768 && bv.max_seq_len > 2 * k && cseg <= 32 * kMaxWords) {
+    const int slot = C == 2 ? 1 : C == 4 ? 2 : 3;
+    if (C > 1 && bv.max_seq_len >= 32768 && bv.max_seq_len > 2 * k && cseg <= 32 * kMaxWords &&
+        ds->cluster_fits[slot]) {
         const int seg = cseg;
         const int cwords = ((seg / 32) + 3) & ~3;
         const int fixed = hist_bytes + kCCand * 8 + 2 * cwords * 4;
-        int stage = (kSmemLimit - kStaticReserve - fixed) / 4 & ~3;
+        int stage = (kMaxDynSmem - fixed) / 4 & ~3;
         if (stage > seg) stage = seg;
         const size_t smem = (size_t)fixed + (size_t)stage * 4;
-        cudaError_t e = cudaFuncSetAttribute(topk_cluster_kernel,
-                                             cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-        if (e != cudaSuccess) return e;
         cudaLaunchConfig_t cfg = {};
         cfg.gridDim = dim3(T * C);
         cfg.blockDim = dim3(kThreads);
@@ -746,57 +805,24 @@ cudaError_t launch_topk(const float* logits, long long ld, const BatchView& bv, 
         attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
         attr[1].val.programmaticStreamSerializationAllowed = 1;
         cfg.attrs = attr;
-        cfg.numAttrs = 1;
-        // whether a cluster of C CTAs fits, asked once per C at the largest shared-memory
-        // size this kernel uses (a smaller request then fits too)
-        static std::atomic<int> fits[4] = {{-1}, {-1}, {-1}, {-1}};   // C = 1, 2, 4, 8
-        const int slot = C == 2 ? 1 : C == 4 ? 2 : 3;
-        int clusters = fits[slot].load(std::memory_order_relaxed);
-        if (clusters < 0) {
-            const int max_smem = kSmemLimit - kStaticReserve;
-            cudaLaunchConfig_t probe = cfg;
-            probe.dynamicSmemBytes = max_smem;
-            int n = 0;
-            e = cudaFuncSetAttribute(topk_cluster_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                     max_smem);
-            if (e == cudaSuccess) e = cudaOccupancyMaxActiveClusters(&n, topk_cluster_kernel, &probe);
-            if (e != cudaSuccess) {
-                (void)cudaGetLastError();
-                n = 0;
-            }
-            clusters = n > 0 ? 1 : 0;
-            fits[slot].store(clusters, std::memory_order_relaxed);
-            e = cudaFuncSetAttribute(topk_cluster_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                     (int)smem);
-            if (e != cudaSuccess) return e;
-        }
-        if (clusters > 0) {
-            cfg.numAttrs = pdl ? 2 : 1;
-            e = cudaLaunchKernelEx(&cfg, topk_cluster_kernel, logits, ld, bv, k, idx, check, cwords,
-                                   stage, row0);
-            if (e != cudaSuccess) return e;
-            return cudaGetLastError();
-        }
-        // no cluster fits: one CTA per row below
+        cfg.numAttrs = pdl ? 2 : 1;
+        cudaError_t e = cudaLaunchKernelEx(&cfg, topk_cluster_kernel, logits, ld, bv, k, idx, check,
+                                           cwords, stage, row0);
+        if (e != cudaSuccess) return e;
+        return cudaGetLastError();
     }
     if (words <= kMaxWords) {
         const int fixed = hist_bytes + kCandCap * 8 + 2 * words * 4;
-        int stage = (kSmemLimit - kStaticReserve - fixed) / 4 & ~3;
+        int stage = (kMaxDynSmem - fixed) / 4 & ~3;
         if (stage > bv.max_seq_len) stage = bv.max_seq_len;
         const size_t smem = (size_t)fixed + (size_t)stage * 4;
-        cudaError_t e = cudaFuncSetAttribute(topk_kernel,
-                                             cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-        if (e != cudaSuccess) return e;
-        e = launch_kernel(topk_kernel, dim3(T), dim3(kThreads), smem, st, pdl, logits, ld,
+        cudaError_t e = launch_kernel(topk_kernel, dim3(T), dim3(kThreads), smem, st, pdl, logits, ld,
                           bv, k, idx, check, words, stage, row0);
         if (e != cudaSuccess) return e;
     } else {
-        const int stage = (kSmemLimit - kStaticReserve - hist_bytes) / 4 & ~3;
+        const int stage = (kMaxDynSmem - hist_bytes) / 4 & ~3;
         const size_t smem = (size_t)hist_bytes + (size_t)stage * 4;
-        cudaError_t e = cudaFuncSetAttribute(topk_long_kernel,
-                                             cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-        if (e != cudaSuccess) return e;
-        e = launch_kernel(topk_long_kernel, dim3(T), dim3(kThreads), smem, st, pdl, logits,
+        cudaError_t e = launch_kernel(topk_long_kernel, dim3(T), dim3(kThreads), smem, st, pdl, logits,
                           ld, bv, k, idx, check, stage, row0);
         if (e != cudaSuccess) return e;
     }

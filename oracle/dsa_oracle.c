@@ -331,11 +331,11 @@ uint16_t oracle_f32_to_bf16(float f) {
  *   slot_mapping  [n]: cache row of token i (page * page_size + row in page);
  *                 a negative entry skips the token
  *   cache_data    [num_rows][dim] of cache_dtype; cache_scale [num_rows] fp32
- * FP8 cache: amax = max_e |x_e| (fp32), scale = amax / 448 in fp32 (1 when
- * amax = 0); the codes use the reciprocal factor inv = 448 / amax (an fp32
- * division, capped at the largest finite fp32 so that a zero or vanishing amax
- * gives zero codes): code_e = e4m3(x_e * inv), the product rounded to fp32.
- * BF16 cache: x rounded to bf16.  FP32 cache: x as is.  The scale
+ * FP8 cache: amax = max_e |x_e| (fp32), scale = amax / 448 rounded to fp32 (1
+ * when amax = 0 or the quotient underflows to 0); code_e = e4m3(x_e / scale),
+ * the quotient an IEEE fp32 division, then rounded to e4m3 (nearest even,
+ * saturating at +-448).  Dequantisation is code * scale, so the codes are x in
+ * units of the scale.  BF16 cache: x rounded to bf16.  FP32 cache: x as is.  The scale
  * of a non-FP8 cache is left untouched.  Returns -1 (after writing the valid
  * tokens) if a slot is >= num_rows.
  */
@@ -356,13 +356,12 @@ int oracle_cache_store(const void* x, int x_dtype, int64_t n, int dim,
             float amax = 0.0f;
             for (int d = 0; d < dim; ++d)
                 if (fabsf(row[d]) > amax) amax = fabsf(row[d]);
-            volatile float scale = amax > 0.0f ? amax / 448.0f : 1.0f;
-            volatile float inv = 448.0f / amax;            /* +inf when amax = 0 */
-            if (inv > FLT_MAX) inv = FLT_MAX;
+            volatile float scale = amax / 448.0f;
+            if (!(scale > 0.0f)) scale = 1.0f;            /* amax = 0 or underflow */
             uint8_t* dst = (uint8_t*)cache_data + slot * dim;
             for (int d = 0; d < dim; ++d) {
-                volatile float product = row[d] * inv;
-                dst[d] = oracle_f32_to_e4m3(product);
+                volatile float quotient = row[d] / scale;
+                dst[d] = oracle_f32_to_e4m3(quotient);
             }
             cache_scale[slot] = scale;
         } else if (cache_dtype == OR_BF16) {

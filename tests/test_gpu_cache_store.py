@@ -135,3 +135,17 @@ def test_stored_kv_feeds_decode_attention():
     H.check_topk(g_idx, g_logits, o_logits, pos, spec.topk)
     o_ref, l_ref = H.oracle_mla(wl, g_idx, rows)
     H.check_mla(out.float().cpu().numpy(), lse.cpu().numpy(), o_ref, l_ref, H.MLA_ATOL_BF16)
+
+
+@pytest.mark.parametrize("dim", [128, 576])
+def test_fp8_codes_on_rounding_boundaries(dim):
+    """Rows whose elements sit next to e4m3 rounding boundaries (see _quant_cases):
+    the last bit of each fp32 quotient x / scale decides the code, so any other way
+    of forming the quotient shows up here as differing bytes."""
+    import _quant_cases as QC
+    x = torch.from_numpy(QC.boundary_rows(300, dim, seed=dim)).cuda()
+    n = x.shape[0]
+    slots = torch.randperm(n + 17, generator=torch.Generator().manual_seed(dim))[:n].cuda()
+    data = torch.zeros(n + 17, dim, dtype=torch.uint8, device="cuda").view(torch.float8_e4m3fn)
+    scale = torch.full((n + 17,), -1.0, device="cuda")
+    _store_and_compare(x, slots.to(torch.int64), data, scale)

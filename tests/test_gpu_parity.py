@@ -11,7 +11,9 @@ import pytest
 import torch
 
 import long_context_sparse_fp8_b200 as L
+from long_context_sparse_fp8_b200 import chunked as CH
 from long_context_sparse_fp8_b200 import workloads as W
+from oracle import oracle as O
 
 import _helpers as H
 
@@ -54,7 +56,7 @@ def test_tiny_prefill_all_rows():
 
 def test_decode_b32_ctx8192():
     wl = _wl("c2", W.decode_b32_8k)
-    _pipeline(wl, H.sample_rows(32, 12, seed=2), decode=True)
+    _pipeline(wl, np.arange(32), decode=True)
 
 
 def test_fused_decode_matches_separate_calls():
@@ -113,18 +115,62 @@ def test_multi_query_decode(nq):
 
 def test_prefill_32k_heavy_hitters():
     wl = _wl("c3", W.prefill_32k)
-    _pipeline(wl, H.sample_rows(wl.spec.total_q, 12, seed=3))
+    _pipeline(wl, H.sample_rows(wl.spec.total_q, 64, seed=3))
 
 
 def test_decode_b64_paged_fp8_kv():
     wl = _wl("c4", W.decode_b64_128k)
-    _pipeline(wl, H.sample_rows(64, 6, seed=4), decode=True)
+    _pipeline(wl, H.sample_rows(64, 8, seed=4), decode=True)
 
 
-@pytest.mark.parametrize("chunk", [0, 15])
-def test_chunked_prefill_128k(chunk):
-    wl = _wl(f"c5-{chunk}", lambda: W.chunked_prefill_128k(chunk))
-    _pipeline(wl, H.sample_rows(wl.spec.total_q, 6, seed=5 + chunk))
+def test_chunked_prefill_128k_whole_prompt():
+    """The whole 131072-token prefill in 16 chunks of 8192, run as the benchmark runs it
+    (per chunk: dsa_cache_store of the chunk's key and latent-KV rows, dsa_indexer_topk,
+    dsa_sparse_mla_prefill).  The caches it wrote must equal the oracle's cache_store of
+    the same rows byte for byte; on chunks 0, 7, 11 and 15, 64 rows each (first, last and
+    62 drawn), the indexer logits, the selection and the attention output are checked
+    against the oracle computed over the oracle's own caches."""
+    _CACHE.clear()
+    torch.cuda.empty_cache()
+    cw = W.make_chunked(W.ChunkedSpec(), device="cuda")
+    s = cw.spec
+    cp = CH.ChunkedPrefill(cw)
+    cp.step()
+    torch.cuda.synchronize()
+    assert L.dsa_device_check() == 0
+    slots = np.arange(s.seq_len, dtype=np.int64)
+    kd, ks = O.cache_store(H.np_bits(cw.k_new), O.BF16, slots,
+                           np.zeros((s.seq_len, s.idx_dim), np.uint8), O.E4M3,
+                           np.zeros(s.seq_len, np.float32))
+    vd, vs = O.cache_store(H.np_bits(cw.kv_new), O.BF16, slots,
+                           np.zeros((s.seq_len, s.d_qk), np.uint8), O.E4M3,
+                           np.zeros(s.seq_len, np.float32))
+    assert np.array_equal(H.np_bits(cw.k_pages).reshape(s.seq_len, -1), kd)
+    assert np.array_equal(H.np_bits(cw.kv), vd)
+    assert np.array_equal(H.np_bits(cw.k_scale).reshape(-1).view(np.uint32), ks.view(np.uint32))
+    assert np.array_equal(H.np_bits(cw.kv_scale).view(np.uint32), vs.view(np.uint32))
+    caches = (torch.from_numpy(kd).cuda().view(W.FP8).reshape(-1, W.INDEXER_PAGE, s.idx_dim),
+              torch.from_numpy(ks).cuda().reshape(-1, W.INDEXER_PAGE),
+              torch.from_numpy(vd).cuda().view(W.FP8), torch.from_numpy(vs).cuda())
+    for c in (0, 7, 11, 15):
+        wl = W.chunk_view(cw, c, *caches)
+        rows = H.sample_rows(s.chunk_q, 64, seed=50 + c)
+        pos = H.positions(wl)[rows]
+        # the chunk's logits from the stand-alone indexer call (the same kernel and row
+        # grouping as the row blocks of dsa_indexer_topk): the selection must be exact on them
+        logits = H.run_indexer(W.chunk_view(cw, c))
+        rows_t = torch.from_numpy(rows).cuda()
+        g_logits = logits[rows_t].cpu().numpy()
+        del logits
+        o_logits = H.oracle_logits(wl, rows)
+        H.check_logits(g_logits, o_logits, pos)
+        g_idx = cp.idx[c][rows_t].cpu().numpy()
+        H.check_topk(g_idx, g_logits, o_logits, pos, s.topk)
+        o_ref, l_ref = H.oracle_mla(wl, g_idx, rows)
+        H.check_mla(cp.out[c][rows_t].float().cpu().numpy(), cp.lse[c][rows_t].cpu().numpy(),
+                    o_ref, l_ref, H.MLA_ATOL_BF16)
+    del cp, cw
+    torch.cuda.empty_cache()
 
 
 @pytest.mark.parametrize("kv_fp8,permute", [(False, False), (True, True)])
@@ -300,3 +346,39 @@ def test_empty_batch_is_a_no_op():
     torch.cuda.synchronize()
     assert L.dsa_device_check() == 0
     assert torch.all(logits == 3.0) and torch.all(idx == 5)
+
+
+def test_back_to_back_fused_decodes_share_a_workspace():
+    """Two dsa_decode calls queued back to back on one stream, the second on a different
+    batch, both keeping their selection in the same workspace: each kernel of the
+    second call waits for the kernel before it before writing anything, so the second
+    call's top-k cannot overwrite the selection the first call's attention still
+    reads.  40 rows (one split, no merge kernel), some shorter than k."""
+    lens_a = [1500, 3000, 900, 4100, 2047, 2048, 2049, 5000] * 5
+    lens_b = [4000, 1200, 2600, 300, 5000, 2100, 64, 3500] * 5
+    wls = [W.make(W.Spec(name=f"b2b{i}", seq_lens=lens, nq=[1] * len(lens), topk=2048,
+                         seed=300 + i), device="cuda")
+           for i, lens in enumerate((lens_a, lens_b))]
+    s = wls[0].spec
+    ref = []
+    for wl in wls:
+        idx = H.run_topk(wl, H.run_indexer(wl))
+        out, lse = H.run_mla(wl, idx, decode=True)
+        ref.append((idx, out, lse))
+    torch.cuda.synchronize()
+    n = max(L.dsa_decode_workspace_size(H.lib_args(wl)[0], s.topk, s.heads, s.d_v) for wl in wls)
+    ws = torch.empty(n, dtype=torch.uint8, device="cuda")
+    for rep in range(3):
+        got = []
+        for wl in wls:
+            batch, kc, kv = H.lib_args(wl)
+            out = torch.empty(s.total_q, s.heads, s.d_v, dtype=torch.bfloat16, device="cuda")
+            lse = torch.empty(s.total_q, s.heads, device="cuda")
+            L.dsa_decode(wl.q_idx, None, wl.w, kc, s.topk, wl.q, kv, batch, s.d_v,
+                         s.softmax_scale, out, lse, None, ws)
+            got.append((out, lse))
+        torch.cuda.synchronize()
+        assert L.dsa_device_check() == 0
+        for (_, r_out, r_lse), (g_out, g_lse) in zip(ref, got):
+            assert torch.equal(r_out, g_out), rep
+            assert torch.equal(r_lse, g_lse), rep

@@ -18,6 +18,7 @@ import pytest
 import torch
 
 from oracle import oracle as O
+import _quant_cases as QC
 
 GOLDEN = os.path.join(os.path.dirname(__file__), "golden")
 
@@ -412,9 +413,9 @@ def _cache(num_rows, dim, dtype):
 def test_cache_store_fp8_scale_codes_and_untouched_rows():
     """scale = amax / 448; the amax element becomes +-448 exactly; every code
     decodes to x / scale within half a code step (1/16 relative, 2^-10 absolute in
-    the subnormal range) plus the fp32 rounding of the factor 448/amax; an all-zero
-    row gets scale 1 and zero codes; rows the slot mapping skips or does not name
-    keep their bytes."""
+    the subnormal range) plus the fp32 rounding of the quotient; an all-zero row gets
+    scale 1 and zero codes; rows the slot mapping skips or does not name keep their
+    bytes."""
     g = np.random.default_rng(10)
     n, dim, rows = 40, 576, 100
     x = g.standard_normal((n, dim)).astype(np.float32)
@@ -445,6 +446,31 @@ def test_cache_store_fp8_scale_codes_and_untouched_rows():
     for r in range(rows):
         if r not in touched:
             assert np.array_equal(data[r], data0[r]) and scale[r] == scale0[r]
+
+
+def test_cache_store_fp8_codes_are_the_rounded_quotient():
+    """The exact codes: e4m3(x / scale) with the quotient an IEEE fp32 division, byte
+    for byte against torch's own fp32 division and float8 cast, on rows whose elements
+    sit next to e4m3 rounding boundaries.  On these rows the quotient's last bit
+    decides the code, so forming it as x * (448 / amax) instead -- or as x * (1/scale)
+    -- changes thousands of codes (checked here too), and the pin fails for either."""
+    x = QC.boundary_rows(48, 576, seed=21)
+    n = x.shape[0]
+    slots = np.arange(n, dtype=np.int64)
+    d0, s0 = _cache(n, 576, O.E4M3)
+    data, scale = O.cache_store(x, O.F32, slots, d0, O.E4M3, s0)
+    amax = np.abs(x).max(axis=1)
+    want_scale = (amax / np.float32(448.0)).astype(np.float32)
+    assert np.array_equal(scale, want_scale)
+    tx = torch.from_numpy(x)
+    want = _bits((tx / torch.from_numpy(want_scale)[:, None]).to(torch.float8_e4m3fn))
+    bad = np.argwhere(data != want)
+    assert bad.size == 0, [(int(i), int(j), float(x[i, j])) for i, j in bad[:5]]
+    inv = torch.from_numpy((np.float32(448.0) / amax).astype(np.float32))[:, None]
+    other = _bits((tx * inv).to(torch.float8_e4m3fn))
+    assert int((other != want).sum()) > 500
+    rcp = torch.from_numpy((np.float32(1.0) / want_scale).astype(np.float32))[:, None]
+    assert int((_bits((tx * rcp).to(torch.float8_e4m3fn)) != want).sum()) > 500
 
 
 def test_cache_store_bf16_and_f32_caches():
