@@ -37,6 +37,7 @@ ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
 
 import long_context_sparse_fp8_b200 as L  # noqa: E402
+from long_context_sparse_fp8_b200 import chunked as CH  # noqa: E402
 from long_context_sparse_fp8_b200 import replicas as R  # noqa: E402
 from long_context_sparse_fp8_b200 import workloads as W  # noqa: E402
 
@@ -44,6 +45,7 @@ METRIC = "DSA tokens/s (decode & prefill) on 1 B200; % of HBM / tensor-core roof
 FLUSH_BYTES = 256 << 20
 
 WORKLOADS = {
+    "chunked_prefill_L131072_16x8192": (W.ChunkedSpec, "chunked"),
     "decode_b32_ctx8192": (W.decode_b32_8k, "decode"),
     "prefill_L32768_q8192": (W.prefill_32k, "prefill"),
     "decode_b64_ctx64k-128k_fp8kv": (W.decode_b64_128k, "decode"),
@@ -59,7 +61,11 @@ def parse():
     p.add_argument("--steps", type=int, default=200)
     p.add_argument("--warmup", type=int, default=10)
     p.add_argument("--impl", choices=["dsa", "reference"], default="dsa")
-    p.add_argument("--workload", choices=sorted(WORKLOADS), default="decode_b32_ctx8192")
+    p.add_argument("--workload", choices=sorted(WORKLOADS),
+                   default="chunked_prefill_L131072_16x8192")
+    p.add_argument("--no-extras", action="store_true",
+                   help="chunked prefill only: skip the decode lines reported beside it")
+    p.add_argument("--no-e2e", action="store_true", help="skip the end-to-end measurement")
     p.add_argument("--no-cpu-baseline", action="store_true")
     p.add_argument("--cpu-seconds", type=float, default=12.0)
     p.add_argument("--fp8-peak", action="store_true",
@@ -331,6 +337,8 @@ def run_dsa(args, rank, world, dev):
     spec_fn, mode = WORKLOADS[args.workload]
     if mode == "store":
         return run_store(args, rank, world, dev)
+    if mode == "chunked":
+        return run_chunked(args, rank, world, dev)
     spec = spec_fn()
     spec.seed = R.replica_seed(spec.seed, rank)  # independent replica inputs per rank
     wl = W.make(spec, device=dev)
@@ -405,7 +413,7 @@ def run_dsa(args, rank, world, dev):
     # independent batches (different seeds, together larger than L2) alternate, so no
     # step finds its inputs in L2 from the step before.
     e2e = None
-    if mode == "decode":
+    if mode == "decode" and not args.no_e2e:
         spec_b = spec_fn()
         spec_b.seed = R.replica_seed(spec.seed + 7, rank)
         sts = [st, Step(W.make(spec_b, device=dev), mode)]
@@ -509,6 +517,272 @@ def run_dsa(args, rank, world, dev):
         "gpu_launches": st.launches_per_step() * args.steps,
         "gpu_launches_note": "fused decode steps in the timed loop (indexer, top-k, attention, merge)",
     }
+
+
+# ----------------------------------------------------------------------------- chunked prefill
+def chunked_work(spec):
+    """Algorithmic work of one whole chunked prefill, per stage: causal (query, key) pairs
+    for the indexer, min(k, pos+1) selected rows per query for the attention."""
+    Lt, k = spec.seq_len, spec.topk
+    n_pairs = Lt * (Lt + 1) // 2
+    n_sel = sum(min(k, t + 1) for t in range(Lt))
+    kv_row = spec.d_qk + 4                                  # fp8 codes + scale
+    store = Lt * (spec.idx_dim * 2 + spec.idx_dim + 4 + 8) + Lt * (spec.d_qk * 2 + spec.d_qk + 4 + 8)
+    return {
+        "store": {"bytes": store, "flops": 0},
+        "indexer": {"flops": 2 * n_pairs * spec.idx_heads * spec.idx_dim},
+        "topk": {"bytes": n_pairs * 4 + Lt * k * 4, "flops": 0},
+        "mla": {"flops": 2 * n_sel * spec.heads * (spec.d_qk + spec.d_v),
+                "bytes": n_sel * (kv_row + 8) + Lt * spec.heads * (spec.d_qk + spec.d_v) * 2},
+        "n_pairs": n_pairs, "n_sel": n_sel,
+    }
+
+
+def run_chunked(args, rank, world, dev):
+    spec = W.ChunkedSpec()
+    spec.seed = R.replica_seed(spec.seed, rank)
+    cw = W.make_chunked(spec, device=dev)
+    cp = CH.ChunkedPrefill(cw)
+    stream = torch.cuda.current_stream()
+    flush = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    for _ in range(max(3, args.warmup)):
+        cp.step()
+    torch.cuda.synchronize()
+    if L.dsa_device_check() != 0:
+        raise RuntimeError("device check recorded an error during warm-up")
+
+    # ---- headline: K whole prefills (16 chunks each)
+    R.barrier(world, dev)
+    with ClockSampler(torch.cuda.current_device()) as clk:
+        step_ms = [sum(x) for x in timed_loop([cp.step], args.steps, flush, stream)]
+    R.barrier(world, dev)
+    ms_max = R.max_over_ranks(statistics.mean(step_ms), world, dev)
+    tokens = spec.seq_len
+    value = R.job_throughput(tokens, ms_max, world)
+
+    # ---- per stage over all chunks: the step's own calls (store, indexer + top-k in
+    # row blocks, attention), then the indexer and the top-k staged through a full logits
+    # buffer, which times the indexer kernel alone
+    R.barrier(world, dev)
+    stage_ms = timed_loop(cp.stages(), args.steps, flush, stream)
+    names = ["store", "select", "mla"]
+    mean_stage = {n: statistics.mean(r[j] for r in stage_ms) for j, n in enumerate(names)}
+    ld = (spec.seq_len + 63) // 64 * 64
+    logits = torch.empty(spec.chunk_q, ld, device=dev)
+    idx_s = torch.empty(spec.chunk_q, spec.topk, dtype=torch.int32, device=dev)
+
+    def staged(which):
+        def f():
+            for c in range(spec.n_chunks):
+                if which == "indexer":
+                    L.dsa_indexer_logits(cw.q_idx[c], None, cw.w[c], cp.kc, cp.batches[c], logits)
+                else:
+                    L.dsa_topk(logits, cp.batches[c], spec.topk, idx_s)
+        return f
+    # the top-k of every chunk reads the last chunk's logits rows (same shape of work)
+    staged("indexer")()
+    sm = timed_loop([staged("indexer"), staged("topk")], max(2, args.steps // 2), flush, stream)
+    R.barrier(world, dev)
+    mean_stage["indexer"] = statistics.mean(r[0] for r in sm)
+    mean_stage["topk"] = statistics.mean(r[1] for r in sm)
+    del logits, idx_s
+    work = chunked_work(spec)
+    hbm_gbs, bf16_tf, peak_kind = measured_peaks()
+    fp8_tf, fp8_src = fp8_peak()
+    ix = work["indexer"]["flops"] / (mean_stage["indexer"] / 1e3) / 1e12
+    mla = work["mla"]["flops"] / (mean_stage["mla"] / 1e3) / 1e12
+    per = {"indexer": {"achieved": round(ix, 1), "peak": fp8_tf, "frac": round(ix / fp8_tf, 4),
+                       "unit": "TFLOP/s", "peak_source": fp8_src},
+           "mla": {"achieved": round(mla, 1), "peak": bf16_tf, "frac": round(mla / bf16_tf, 4),
+                   "unit": "TFLOP/s", "peak_source": f"{peak_kind} (burst bf16)"}}
+    dom = "indexer" if mean_stage["indexer"] >= mean_stage["mla"] else "mla"
+    kernel_file = {"indexer": "indexer_tc.cu", "mla": "mla_tc.cu"}[dom]
+    roof = {"bound": "tensor", **per[dom], "kernel": dom,
+            "traffic": ncu_traffic(args.workload, kernel_file),
+            "indexer_fp8": per["indexer"], "mla_bf16": per["mla"],
+            "stage_ms": {n: round(v, 3) for n, v in mean_stage.items()},
+            "stage_note": "store / select (indexer + top-k in row blocks) / mla are the step's "
+                          "calls over all 16 chunks; indexer and topk are the same work staged "
+                          "through a full logits buffer",
+            "flops_per_step": {"indexer": work["indexer"]["flops"], "mla": work["mla"]["flops"]},
+            "store": {"achieved_gbs": round(work["store"]["bytes"] / (mean_stage["store"] / 1e3)
+                                            / 1e9, 1), "peak": hbm_gbs}}
+
+    # ---- end to end through host buffers: every chunk's inputs (new key / KV rows, slot
+    # maps, q_idx, w, q) are uploaded from pinned host memory and its output o is read
+    # back; the uploads of chunk c+1 and the download of chunk c-1 overlap chunk c on two
+    # copy streams (two device input sets and two pinned output buffers alternate)
+    e2e = None
+    if not args.no_e2e:
+        try:
+            e2e = _chunked_e2e(args, cw, cp, stream, world, dev, tokens)
+        except RuntimeError as ex:   # e.g. pinned host memory unavailable
+            torch.cuda.synchronize(dev)
+            e2e = {"value": None, "unit": "tokens/s", "h2d_bytes_per_step": 0,
+                   "d2h_bytes_per_step": 0, "error": str(ex)[:200]}
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        cpu = chunked_cpu_baseline(cw, args.cpu_seconds)
+    if L.dsa_device_check() != 0:
+        raise RuntimeError("device check recorded an error in the timed region")
+    launches = cp.launches_per_step()
+    res = {
+        "metric": METRIC, "value": round(value, 1), "unit": "tokens/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms_max, 4),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "fp8 e4m3 (indexer, latent KV cache) + bf16 q (MLA), fp32 accumulate",
+        "data": "synthetic (seeded N(0,1) key / latent-KV rows and queries)",
+        "config": {"workload": spec.name, "mode": "chunked prefill", "context": spec.seq_len,
+                   "chunks": spec.n_chunks, "chunk_queries": spec.chunk_q, "topk": spec.topk,
+                   "indexer": f"fp8 e4m3 {spec.idx_heads}x{spec.idx_dim}, page 64, per-token "
+                              "scale (written by dsa_cache_store each chunk)",
+                   "mla": f"{spec.heads} heads, d_qk {spec.d_qk}, d_v {spec.d_v}, fp8 latent "
+                          "KV page 1 (written by dsa_cache_store each chunk)",
+                   "step": "per chunk: dsa_cache_store x2, dsa_indexer_topk, "
+                           "dsa_sparse_mla_prefill",
+                   "l2": "flushed between steps (256 MiB write); the inputs (~21 GB) exceed L2",
+                   "sparse_attention_ratio": round(work["n_sel"] / work["n_pairs"], 5),
+                   "parallelism": f"replicas x{world}"},
+        "roofline": roof, "cpu_baseline": cpu, "e2e": e2e, "clocks": clk.summary(),
+        "gpu_launches": launches * args.steps,
+        "gpu_launches_note": f"{launches} launches per whole prefill (per chunk: 2 stores, "
+                             "indexer and top-k per row block, attention)",
+    }
+    del cp, cw
+    torch.cuda.empty_cache()
+    if not args.no_extras:
+        res["extra"] = {}
+        for wname in ("decode_b32_ctx8192", "decode_b64_ctx64k-128k_fp8kv"):
+            sub = argparse.Namespace(**vars(args))
+            sub.workload, sub.no_cpu_baseline, sub.no_e2e = wname, True, True
+            r = run_dsa(sub, rank, world, dev)
+            res["extra"][wname] = {k: r[k] for k in ("value", "unit", "ms_per_step", "config")}
+            rf = r["roofline"]
+            res["extra"][wname]["roofline"] = {k: rf.get(k) for k in (
+                "bound", "kernel", "achieved", "peak", "unit", "frac", "stage_ms")}
+            res["extra"][wname]["clocks"] = r["clocks"]
+            res["gpu_launches"] += r["gpu_launches"]
+            torch.cuda.empty_cache()
+        res["gpu_launches_note"] += "; plus the two decode lines under 'extra'"
+    return res
+
+
+def _chunked_e2e(args, cw, cp, stream, world, dev, tokens):
+    s = cw.spec
+    C = s.n_chunks
+    names = ("k_new", "kv_new", "k_slots", "kv_slots")
+    host = {n: [getattr(cw, n)[cp.rows(c)].cpu().pin_memory() for c in range(C)] for n in names}
+    for n in ("q_idx", "w", "q"):
+        host[n] = [getattr(cw, n)[c].cpu().pin_memory() for c in range(C)]
+    dev_in = [{n: torch.empty_like(host[n][0], device=dev) for n in host} for _ in range(2)]
+    out_host = [torch.empty(cp.out.shape[1:], dtype=cp.out.dtype).pin_memory() for _ in range(2)]
+    h2d_s, d2h_s = torch.cuda.Stream(dev), torch.cuda.Stream(dev)
+    ev = lambda: torch.cuda.Event()  # noqa: E731
+    in_ready, comp_done, out_free = [ev(), ev()], [ev(), ev()], [ev(), ev()]
+
+    def run(n_steps, cs):
+        i = 0
+        for _ in range(n_steps):
+            for c in range(C):
+                b = i & 1
+                d = dev_in[b]
+                with torch.cuda.stream(h2d_s):
+                    if i >= 2:
+                        h2d_s.wait_event(comp_done[b])   # chunk i-2 done with this input set
+                    for n in host:
+                        d[n].copy_(host[n][c], non_blocking=True)
+                    in_ready[b].record(h2d_s)
+                cs.wait_event(in_ready[b])
+                if i >= 2:
+                    cs.wait_event(out_free[b])          # output of chunk i-2 read back
+                cp.store(c, d["k_new"], d["kv_new"], d["k_slots"], d["kv_slots"], stream=cs)
+                cp.select(c, d["q_idx"], d["w"], cp.idx[b], stream=cs)
+                cp.attend(c, d["q"], cp.idx[b], cp.out[b], cp.lse[b], stream=cs)
+                comp_done[b].record(cs)
+                with torch.cuda.stream(d2h_s):
+                    d2h_s.wait_event(comp_done[b])
+                    out_host[b].copy_(cp.out[b], non_blocking=True)
+                    out_free[b].record(d2h_s)
+                i += 1
+        for e in out_free:
+            cs.wait_event(e)
+
+    h2d_s.wait_stream(stream)
+    d2h_s.wait_stream(stream)
+    run(1, stream)
+    torch.cuda.synchronize(dev)
+    R.barrier(world, dev)
+    n_steps = max(1, min(args.steps, 5))
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    h2d_s.wait_stream(stream)
+    d2h_s.wait_stream(stream)
+    e0.record(stream)
+    run(n_steps, stream)
+    e1.record(stream)
+    torch.cuda.synchronize(dev)
+    e_ms = R.max_over_ranks(e0.elapsed_time(e1) / n_steps, world, dev)
+    h2d = sum(t.numel() * t.element_size() for n in host for t in host[n])
+    d2h = C * out_host[0].numel() * out_host[0].element_size()
+    return {"value": round(R.job_throughput(tokens, e_ms, world), 1), "unit": "tokens/s",
+            "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": round(e_ms, 3),
+            "steps": n_steps,
+            "method": "per chunk: pinned H2D of the new key / latent-KV rows, slot maps, q_idx, "
+                      "w and q, D2H of o; the next chunk's uploads and the previous chunk's "
+                      "download overlap the chunk on two copy streams; eager launches"}
+
+
+def _chunked_oracle_setup(cw):
+    """The oracle's own FP8 caches for the whole prompt (its cache_store on the rows), as
+    the inputs of its per-row indexer and attention."""
+    import numpy as np
+    from oracle import oracle as O
+    s = cw.spec
+    kx = cw.k_new.view(torch.int16).cpu().numpy().view(np.uint16)
+    vx = cw.kv_new.view(torch.int16).cpu().numpy().view(np.uint16)
+    slots = np.arange(s.seq_len, dtype=np.int64)
+    kd, ks = O.cache_store(kx, O.BF16, slots, np.zeros((s.seq_len, s.idx_dim), np.uint8), O.E4M3,
+                           np.zeros(s.seq_len, np.float32))
+    vd, vs = O.cache_store(vx, O.BF16, slots, np.zeros((s.seq_len, s.d_qk), np.uint8), O.E4M3,
+                           np.zeros(s.seq_len, np.float32))
+    dev = cw.device
+    return (torch.from_numpy(kd).to(dev).view(W.FP8).reshape(-1, W.INDEXER_PAGE, s.idx_dim),
+            torch.from_numpy(ks).to(dev).reshape(-1, W.INDEXER_PAGE),
+            torch.from_numpy(vd).to(dev).view(W.FP8), torch.from_numpy(vs).to(dev))
+
+
+def _chunked_oracle_rows(cw, caches, positions):
+    """Oracle indexer + top-k + attention for the query rows at the given prompt positions."""
+    import numpy as np
+    s = cw.spec
+    for c in np.unique(positions // s.chunk_q):
+        rows = positions[positions // s.chunk_q == c] - c * s.chunk_q
+        wl = W.chunk_view(cw, int(c), *caches)
+        _oracle_rows(wl, "prefill", rows)
+
+
+def chunked_cpu_baseline(cw, seconds):
+    """The oracle on prompt positions drawn uniformly from the whole prompt (so rows/s
+    estimates the whole prefill's tokens/s), sized to about `seconds` of work."""
+    import numpy as np
+    from oracle import oracle as O
+    s = cw.spec
+    caches = _chunked_oracle_setup(cw)
+    t0 = time.perf_counter()
+    _chunked_oracle_rows(cw, caches, np.array([s.seq_len // 2]))
+    one = time.perf_counter() - t0
+    threads = O.num_threads()
+    n = int(max(2, min(256, seconds / max(one, 1e-3) * threads)))
+    pos = np.sort(np.random.default_rng(0).choice(s.seq_len, n, replace=False))
+    t0 = time.perf_counter()
+    _chunked_oracle_rows(cw, caches, pos)
+    dt = time.perf_counter() - t0
+    return {"value": round(len(pos) / dt, 3), "unit": "tokens/s", "cores": threads,
+            "kind": "oracle",
+            "sample": f"{len(pos)} query rows at uniformly drawn positions of the "
+                      f"{s.seq_len}-token prompt (indexer + top-k + MLA per row, fp64, over the "
+                      f"oracle's own FP8 caches), {dt:.1f} s; rows/s estimates the whole "
+                      "prefill's tokens/s"}
 
 
 # ----------------------------------------------------------------------------- cache writes
@@ -679,6 +953,8 @@ def run_reference(args, rank, world):
     dev = "cuda" if torch.cuda.is_available() else "cpu"
     if mode == "store":
         return _store_reference(args, world, dev)
+    if mode == "chunked":
+        return _chunked_reference(args, world, dev)
     spec = spec_fn()
     wl = W.make(spec, device=dev)
     T = spec.total_q
@@ -708,6 +984,47 @@ def run_reference(args, rank, world):
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
         "dtype": "f64", "data": "synthetic (seeded N(0,1) caches and queries)",
         "config": {"workload": spec.name, "mode": mode, "queries": T, "topk": spec.topk},
+        "cpu_baseline": {"kind": "oracle", "cores": threads, "sample": sample,
+                         "value": round(value, 3), "unit": "tokens/s"},
+        "e2e": {"value": round(value, 3), "unit": "tokens/s", "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }
+
+
+def _chunked_reference(args, world, dev):
+    import numpy as np
+    from oracle import oracle as O
+    spec = W.ChunkedSpec()
+    cw = W.make_chunked(spec, device=dev)
+    caches = _chunked_oracle_setup(cw)
+    t0 = time.perf_counter()
+    _chunked_oracle_rows(cw, caches, np.array([spec.seq_len // 2]))
+    one = time.perf_counter() - t0
+    threads = O.num_threads()
+    budget = 150.0 / max(1, args.steps + args.warmup)
+    per_step = int(max(1, min(256, budget / max(one, 1e-3) * threads)))
+    rng = np.random.default_rng(0)
+    draw = lambda: np.sort(rng.choice(spec.seq_len, per_step, replace=False))  # noqa: E731
+    for _ in range(args.warmup):
+        _chunked_oracle_rows(cw, caches, draw())
+    times = []
+    for _ in range(args.steps):
+        pos = draw()
+        t0 = time.perf_counter()
+        _chunked_oracle_rows(cw, caches, pos)
+        times.append(time.perf_counter() - t0)
+    ms = statistics.mean(times) * 1e3
+    value = per_step / (ms / 1e3)
+    sample = (f"{per_step} query rows per step at uniformly drawn positions of the "
+              f"{spec.seq_len}-token prompt (indexer + top-k + MLA, fp64); rows/s estimates "
+              "the whole prefill's tokens/s")
+    return {
+        "impl": "reference", "metric": METRIC, "value": round(value, 3), "unit": "tokens/s",
+        "n_gpus": world, "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms, 3),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic (seeded N(0,1) key / latent-KV rows and queries)",
+        "config": {"workload": spec.name, "mode": "chunked prefill", "context": spec.seq_len,
+                   "chunks": spec.n_chunks, "topk": spec.topk},
         "cpu_baseline": {"kind": "oracle", "cores": threads, "sample": sample,
                          "value": round(value, 3), "unit": "tokens/s"},
         "e2e": {"value": round(value, 3), "unit": "tokens/s", "h2d_bytes_per_step": 0,

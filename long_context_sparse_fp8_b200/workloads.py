@@ -331,3 +331,112 @@ def store_prompt_128k(seed: int = 1240) -> StoreSpec:
     """A 131072-token prompt's keys and latent KV written into FP8 caches at once
     (bf16 rows in; page-64 key cache and page-1 KV cache, fragmented)."""
     return StoreSpec(name="store_L131072_fp8", n_tokens=131072, seed=seed)
+
+
+# ----------------------------------------------------------------------------------------
+# The whole chunked prefill: one sequence of n_chunks x chunk_q tokens, processed chunk by
+# chunk against the growing causal prefix.  Each chunk brings its tokens' new indexer-key
+# and latent-KV rows (written into the FP8 caches before the chunk is scored) and its
+# queries.
+
+@dataclass
+class ChunkedSpec:
+    """A prompt of ``n_chunks * chunk_q`` tokens prefilled in chunks of ``chunk_q``."""
+    name: str = "chunked_prefill_L131072_16x8192"
+    n_chunks: int = 16
+    chunk_q: int = 8192
+    topk: int = 2048
+    idx_heads: int = 64
+    idx_dim: int = 128
+    w_std: float = 1.0 / 8.0
+    heads: int = 128
+    d_qk: int = 576
+    d_v: int = 512
+    softmax_scale: float = 1.0 / math.sqrt(192.0)
+    seed: int = 1239
+
+    @property
+    def seq_len(self) -> int:
+        return self.n_chunks * self.chunk_q
+
+    def chunk_spec(self, c: int) -> Spec:
+        """The shape of chunk c as a one-sequence Spec (queries = its chunk_q tokens)."""
+        return Spec(name=f"{self.name}_chunk{c}", seq_lens=[self.chunk_q * (c + 1)],
+                    nq=[self.chunk_q], topk=self.topk, idx_heads=self.idx_heads,
+                    idx_dim=self.idx_dim, w_std=self.w_std, heads=self.heads, d_qk=self.d_qk,
+                    d_v=self.d_v, kv_fp8=True, softmax_scale=self.softmax_scale,
+                    seed=self.seed)
+
+
+@dataclass
+class ChunkedWorkload:
+    spec: ChunkedSpec
+    k_new: torch.Tensor            # [L, d_I] bf16: every token's indexer key row
+    kv_new: torch.Tensor           # [L, 576] bf16: every token's latent-KV row
+    k_slots: torch.Tensor          # [L] int64: page * 64 + row (identity table)
+    kv_slots: torch.Tensor         # [L] int64 slot (identity table)
+    k_pages: torch.Tensor          # [L/64, 64, d_I] fp8, filled chunk by chunk
+    k_scale: torch.Tensor          # [L/64, 64] fp32
+    k_block_table: torch.Tensor    # [1, L/64] int32
+    kv: torch.Tensor               # [L, 576] fp8, filled chunk by chunk
+    kv_scale: torch.Tensor         # [L] fp32
+    kv_slot_table: torch.Tensor    # [1, L] int32
+    q_idx: torch.Tensor            # [n_chunks, chunk_q, H_I, d_I] fp8
+    w: torch.Tensor                # [n_chunks, chunk_q, H_I] fp32
+    q: torch.Tensor                # [n_chunks, chunk_q, heads, 576] bf16
+    cu_q: torch.Tensor             # [2] int32: (0, chunk_q)
+    seq_lens: torch.Tensor         # [n_chunks] int32: chunk_q * (c + 1)
+
+    @property
+    def device(self):
+        return self.q.device
+
+
+def make_chunked(spec: ChunkedSpec, device="cpu") -> ChunkedWorkload:
+    """Draw the chunked prefill (seeded N(0,1) rows and queries; caches start empty, with a
+    marker byte, and identity page / slot tables)."""
+    device = torch.device(device)
+    g = torch.Generator(device=device).manual_seed(spec.seed + 1)
+    Lt, C, Q = spec.seq_len, spec.n_chunks, spec.chunk_q
+    if Lt % INDEXER_PAGE:
+        raise ValueError("the prompt length must be a multiple of the indexer page (64)")
+    n_pages = Lt // INDEXER_PAGE
+    k_new = torch.randn(Lt, spec.idx_dim, generator=g, device=device).to(torch.bfloat16)
+    kv_new = torch.randn(Lt, spec.d_qk, generator=g, device=device).to(torch.bfloat16)
+    pos = torch.arange(Lt, device=device, dtype=torch.int64)
+    q_idx = torch.empty(C, Q, spec.idx_heads, spec.idx_dim, dtype=FP8, device=device)
+    w = torch.empty(C, Q, spec.idx_heads, device=device)
+    q = torch.empty(C, Q, spec.heads, spec.d_qk, dtype=torch.bfloat16, device=device)
+    for c in range(C):          # one chunk at a time bounds the fp32 temporaries
+        q_idx[c] = torch.randn(Q, spec.idx_heads, spec.idx_dim, generator=g,
+                               device=device).clamp(-FP8_MAX, FP8_MAX).to(FP8)
+        w[c] = torch.randn(Q, spec.idx_heads, generator=g, device=device) * spec.w_std
+        q[c] = torch.randn(Q, spec.heads, spec.d_qk, generator=g, device=device).to(torch.bfloat16)
+    marker = 0x5A
+    return ChunkedWorkload(
+        spec=spec, k_new=k_new, kv_new=kv_new, k_slots=pos.clone(), kv_slots=pos.clone(),
+        k_pages=torch.full((n_pages, INDEXER_PAGE, spec.idx_dim), marker, dtype=torch.uint8,
+                           device=device).view(FP8),
+        k_scale=torch.full((n_pages, INDEXER_PAGE), -1.0, device=device),
+        k_block_table=torch.arange(n_pages, dtype=torch.int32, device=device).reshape(1, -1),
+        kv=torch.full((Lt, spec.d_qk), marker, dtype=torch.uint8, device=device).view(FP8),
+        kv_scale=torch.full((Lt,), -1.0, device=device),
+        kv_slot_table=torch.arange(Lt, dtype=torch.int32, device=device).reshape(1, -1),
+        q_idx=q_idx, w=w, q=q,
+        cu_q=torch.tensor([0, Q], dtype=torch.int32, device=device),
+        seq_lens=torch.tensor([Q * (c + 1) for c in range(C)], dtype=torch.int32, device=device))
+
+
+def chunk_view(cw: ChunkedWorkload, c: int, k_pages=None, k_scale=None, kv=None,
+               kv_scale=None) -> Workload:
+    """Chunk c of a chunked prefill as a one-sequence Workload over the whole caches (the
+    cache tensors may be replaced, e.g. by copies written elsewhere)."""
+    s = cw.spec.chunk_spec(c)
+    return Workload(spec=s, cu_q=cw.cu_q, seq_lens=cw.seq_lens[c:c + 1].contiguous(),
+                    q_idx=cw.q_idx[c], w=cw.w[c],
+                    k_pages=cw.k_pages if k_pages is None else k_pages,
+                    k_scale=cw.k_scale if k_scale is None else k_scale,
+                    k_block_table=cw.k_block_table, q=cw.q[c],
+                    kv=cw.kv if kv is None else kv,
+                    kv_scale=cw.kv_scale if kv_scale is None else kv_scale,
+                    kv_slot_table=cw.kv_slot_table)
