@@ -85,6 +85,10 @@ typedef enum dsa_dtype {
 #define DSA_CHECK_BAD_INDEX 2        /* top-k index outside [-1, pos] */
 #define DSA_CHECK_BAD_BATCH 3        /* nq_b > seq_lens[b], seq_lens[b] > max_seq_len, ... */
 #define DSA_CHECK_TIMEOUT 4          /* a bounded on-chip wait gave up */
+#define DSA_CHECK_FP16_RANGE 5       /* the tensor-core attention met a bf16 query or
+                                        latent-KV value of magnitude > 65504 (or a
+                                        non-finite one): its fp16 operands saturate
+                                        there, so that output is not exact */
 
 /* A ragged batch of sequences.  Host fields are upper bounds used to size
  * grids and check strides; device arrays are read by the kernels. */

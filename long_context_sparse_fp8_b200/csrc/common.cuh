@@ -12,7 +12,7 @@ namespace dsa {
 enum DType : int { kF32 = 0, kBF16 = 1, kE4M3 = 2 };
 
 enum CheckCode : int { kCheckNone = 0, kCheckBadPage = 1, kCheckBadIndex = 2, kCheckBadBatch = 3,
-                       kCheckTimeout = 4 };
+                       kCheckTimeout = 4, kCheckFp16Range = 5 };
 
 // Plain copies of the ABI structs passed to kernels by value.
 struct BatchView {

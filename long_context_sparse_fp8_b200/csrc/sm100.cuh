@@ -80,11 +80,11 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, int* c
 // Warp-wide wait: every lane tests the barrier (one warp instruction, a broadcast
 // read) and the warp reconverges before returning -- about 60 cycles on a completed
 // phase, against ~190 for polling from one lane and broadcasting the result.  Must
-// be called by all 32 lanes.
+// be called by all 32 lanes; the result is the same on every lane (a lane that gave
+// up fails the wait for the whole warp), so callers branch on it without diverging.
 __device__ __forceinline__ bool mbar_wait_warp(uint64_t* bar, uint32_t parity, int* check) {
     const bool ok = mbar_try_wait(bar, parity) || mbar_wait(bar, parity, check);
-    __syncwarp();
-    return ok;
+    return __all_sync(0xffffffffu, ok);
 }
 
 // ---------------------------------------------------------------- clusters

@@ -175,14 +175,6 @@ def sparse_mla(q, q_dtype, heads, d_qk, d_v, softmax_scale, kv, kv_dtype, kv_sca
     return out, lse
 
 
-def decode(idx_args: dict, k: int, mla_args: dict, cu_q, seq_lens, ld, rows=None):
-    """Fused decode = indexer logits -> top-k -> sparse MLA, on the same rows."""
-    logits = indexer_logits(cu_q=cu_q, seq_lens=seq_lens, ld=ld, rows=rows, **idx_args)
-    sel = topk(logits, cu_q, seq_lens, k, rows=rows)
-    out, lse = sparse_mla(cu_q=cu_q, seq_lens=seq_lens, idx=sel, rows=rows, **mla_args)
-    return logits, sel, out, lse
-
-
 def f32_to_e4m3(x: float) -> int:
     """One fp32 value to its e4m3 code (RNE, saturating at 448, sign kept)."""
     return int(_load().oracle_f32_to_e4m3(float(x)))

@@ -382,3 +382,31 @@ def test_back_to_back_fused_decodes_share_a_workspace():
         for (_, r_out, r_lse), (g_out, g_lse) in zip(ref, got):
             assert torch.equal(r_out, g_out), rep
             assert torch.equal(r_lse, g_lse), rep
+
+
+@pytest.mark.parametrize("where", ["kv", "q"])
+def test_fp16_range_is_reported(where):
+    """The tensor-core attention computes on fp16 operands: a bf16 latent-KV row or query
+    with entries beyond +-65504 cannot be represented there, and the call must say so
+    (DSA_CHECK_FP16_RANGE) instead of returning silently saturated results.  Rows of
+    ordinary magnitude in the same call are still exact."""
+    spec = W.Spec(name="range", seq_lens=[3000, 2500], nq=[3, 2], topk=2048, seed=91)
+    wl = W.make(spec, device="cuda")
+    if where == "kv":
+        wl.kv[17, :8] = 1.0e5                      # slot 17 = position 17 of sequence 0
+        wl.kv[18, 100] = -2.0e5
+    else:
+        wl.q[1, 5, 7] = 1.0e5
+    idx = torch.arange(spec.topk, dtype=torch.int32, device="cuda").repeat(spec.total_q, 1)
+    pos = torch.from_numpy(H.positions(wl)).cuda()
+    idx = torch.where(idx <= pos[:, None], idx, torch.full_like(idx, -1))
+    assert L.dsa_device_check() == 0
+    out, lse = H.run_mla(wl, idx)
+    torch.cuda.synchronize()
+    assert L.dsa_device_check(reset=True) == 5     # DSA_CHECK_FP16_RANGE
+    assert L.dsa_device_check() == 0
+    # the rows of sequence 1 see neither the large KV rows nor the large query value
+    rows = np.array([3, 4])
+    o_ref, l_ref = H.oracle_mla(wl, idx.cpu().numpy()[rows], rows)
+    H.check_mla(out[3:5].float().cpu().numpy(), lse[3:5].cpu().numpy(), o_ref, l_ref,
+                H.MLA_ATOL_BF16)
