@@ -8,33 +8,41 @@
 // KV cache: "DeepSeek V3.2 usage guide", attention-kernel section; 128 heads,
 // 576 = 512 latent + 64 rope, V = the 512 latent columns).
 //
-// Why two CTAs per query.  The fp32 output tile O (128 heads x 512) would fill all
-// 512 TMEM columns of an SM, leaving no room for the scores.  So CTA v (v = 0, 1)
-// of a (query, split) owns V columns [256v, 256v+256): it computes the full score
-// tile S = Q . KV^T (K = 576) itself, runs the softmax, and accumulates its half of
-// O.  The two CTAs repeat the QK product (1.5x the unique tensor work) but never
-// talk to each other: exchanging partial score tiles through distributed shared
-// memory moves only ~8 bytes per cycle between a CTA pair, slower than recomputing.
+// One (query, split) runs on a pair of SMs: a cluster of two CTAs whose tensor cores
+// act as one (tcgen05 cta_group::2, issued by the even CTA).  The fp32 output tile O
+// (128 heads x 512) needs all 512 TMEM columns of one SM, so it is split by heads:
+// CTA r holds heads [64r, 64r+64).  A tile of 64 selected keys is split by keys: CTA r
+// gathers keys [32r, 32r+32) of the tile, whole rows, into its shared memory, and the
+// paired MMA  S = Q . K^T  (M = 128 heads over the pair, N = 64 keys, K = 576) reads each
+// CTA's query rows and both CTAs' key halves, so every selected row enters one SM for
+// the scores.  For O += P . V (M = 128, N = 2 x 256 V dims, K = 64 keys) each CTA
+// supplies half of the N columns -- V dims {128r..128r+127, 256+128r..+127} -- for all
+// 64 keys, so it also gathers those 512 bytes of the peer's 32 rows (1.44x the
+// algorithmic bytes into the SMs, against 2x when each SM of a pair gathers every row).
 //
-// Roles (352 threads): warps 0-3 = softmax (thread = head = TMEM lane), warps 4-9 =
-// gather (3 threads per selected row), warp 10 = TMEM owner and MMA issuer.  The
-// gather runs a per-thread pipeline over tiles: the index of tile j+5, the slot of
-// tile j+4 and an L2 prefetch of the rows of tile j+2 are in flight while tile j is
-// copied.  bf16 rows go to shared memory by asynchronous 16-byte copies (no register
-// staging); e4m3 rows are loaded one tile ahead into registers and converted to bf16
-// (exact).  S = Q.K^T runs on bf16 operands.  P is kept in fp16 (11 significant
-// bits; bf16 P loses up to 2^-9 relative per term, too much for rows dominated by a
-// few large values), so once S_j has read a tile, the gather group converts this
-// CTA's V columns of it in place from bf16 to fp16 (exact for magnitudes in
-// [2^-14, 65504]; larger ones saturate) while the softmax runs, and P.V runs on fp16.
+// Operands are fp16: the query and the rows are converted on the way into shared memory
+// (bf16 -> fp16 is exact for magnitudes in [2^-14, 65504]; smaller ones keep an
+// absolute precision of 2^-24, larger or non-finite ones saturate and are reported as
+// DSA_CHECK_FP16_RANGE; e4m3 -> fp16 is always exact), so S and P.V take the same
+// operands and P keeps 11 significant bits (bf16 P loses too many for rows dominated by
+// a few large values).  FP8 rows keep their codes; the per-row scale multiplies S and P
+// in fp32.
 //
-// Tensor memory: O_v (256 columns), two 64-column score buffers (S_j in fp32, then
-// P_j in fp16 written over it, so S_{j+1} never waits for the softmax of tile j) and query dims 0..255 (128 columns); dims 256..575 of the query sit in shared memory
-// next to a 2-stage ring of gathered 64-row tiles (72 KB each, 128-byte swizzled
-// K-major regions of 64 dims).  Per tile: 36 MMAs (M=128, N=64, K=16) for S -- A
-// from TMEM or shared memory -- and 4 MMAs (M=128, N=256, K=16) for P.V_v with A =
-// P in TMEM.  Online softmax in base 2 with lazy rescaling (O and l are
-// rescaled only when the running max grows by more than 2^8).
+// Tensor memory, per CTA (both CTAs allocate the same 512 columns; the paired MMA
+// writes each CTA's rows into its own TMEM): O at columns 0..255 (lanes 0-63 hold dims
+// {0..127, 256..383} of heads 0..63 of this CTA, lanes 64-127 dims {128..255,
+// 384..511}); two score buffers of 32 columns (lanes 0-63: keys 0..31 of the tile,
+// lanes 64-127: keys 32..63); query dims 0..383 at columns 320..511, each head's row
+// held twice (lanes h and h+64), the A layout of a paired MMA with A in TMEM.  Query
+// dims 384..575 stay in shared memory.
+//
+// Roles (416 threads per CTA): warps 0-3 = softmax (thread = TMEM lane: head h = lane %
+// 64, key half lane / 64; the two threads of a head exchange row maxima through shared
+// memory); warps 4-11 = gather, two groups of four warps, group g filling stage g with
+// tiles g, g+2, ... (a stage = this CTA's 32 key rows, 36 KB, + the V block of all 64
+// keys, 32 KB); warp 12 = TMEM owner and, in the even CTA, the MMA issuer.  Online
+// softmax in base 2 with lazy rescaling (O and l are rescaled only when the running
+// max grows by more than 2^8).
 #include <climits>
 
 #include "kernels.h"
@@ -46,38 +54,39 @@ namespace {
 using namespace sm100;
 
 constexpr int kHeads = 128;
-constexpr int kTile = 64;
-constexpr int kThreads = 352;
+constexpr int kTile = 64;                 // keys per tile (32 per CTA)
+constexpr int kThreads = 416;
 constexpr int kGatherWarp0 = 4;
-constexpr int kGatherThreads = 192;    // two groups of 96, one per KV stage
-constexpr int kGroupThreads = 96;
-constexpr int kMmaWarp = 10;
-
+constexpr int kGroupThreads = 128;
+constexpr int kMmaWarp = 12;
 constexpr int kStages = 2;
-constexpr int kRegions = 9;                              // 64-dim regions of a 576-dim row
-constexpr uint32_t kQsRegions = 5;                       // query dims 256..575 in smem
-constexpr uint32_t kQsBytes = kQsRegions * 16384;        // 128 rows x 128 B per region
-constexpr uint32_t kStageBytes = kRegions * 8192;        // 64 rows x 128 B per region
+
+constexpr uint32_t kQsBytes = 3 * 8192;                  // query dims 384..575, 64 rows
+constexpr uint32_t kPBytes = 8192;                       // P: 64 heads x 64 keys fp16
+constexpr uint32_t kSbufBytes = 9 * 4096;                // 32 rows x 9 regions of 64 dims
+constexpr uint32_t kVblkBytes = 4 * 8192;                // 64 keys x 4 blocks of 64 V dims
+constexpr uint32_t kStageBytes = kSbufBytes + kVblkBytes;
 constexpr uint32_t kOffQs = 0;
-constexpr uint32_t kOffKV = kOffQs + kQsBytes;
-constexpr uint32_t kOffFlag = kOffKV + kStages * kStageBytes;   // [stage][64] validity bytes
-constexpr uint32_t kOffScale = kOffFlag + kStages * 64;         // [stage][64] fp32 kv scale
-constexpr uint32_t kOffSlot = kOffScale + kStages * 256;       // [stage][64] int slot
-constexpr uint32_t kOffBar = kOffSlot + kStages * 256;
-constexpr uint32_t kNumBars = 16;
+constexpr uint32_t kOffP = kOffQs + kQsBytes;
+constexpr uint32_t kOffStage = kOffP + 2 * kPBytes;
+constexpr uint32_t kOffSlot = kOffStage + kStages * kStageBytes;   // [stage][64] int
+constexpr uint32_t kOffScale = kOffSlot + kStages * 256;           // [stage][64] fp32
+constexpr uint32_t kOffRed = kOffScale + kStages * 256;            // [3][128] fp32
+constexpr uint32_t kOffRing = kOffRed + 3 * 128 * 4;              // [4][64] int slots
+constexpr uint32_t kOffRingSc = kOffRing + 4 * 256;                // [4][64] fp32 scales
+constexpr uint32_t kOffBar = kOffRingSc + 4 * 256;
+constexpr uint32_t kNumBars = 23;
 constexpr uint32_t kSmemBytes = kOffBar + kNumBars * 8 + 16 + 1024;
 static_assert(kSmemBytes <= 232448, "shared memory budget");
+static_assert(kStageBytes % 1024 == 0 && kOffStage % 1024 == 0, "swizzled tiles need 1 KB alignment");
 
 constexpr uint32_t kTmemCols = 512;
-constexpr uint32_t kColO = 0;      // 256 output columns
-constexpr uint32_t kColS = 256;    // two 64-column buffers: S_j (fp32), then P_j (fp16,
-                                   // 32 columns) over it
-constexpr uint32_t kColQ = 384;    // 128 columns = query dims 0..255 as bf16 pairs
-constexpr int kQtSteps = 16;       // K-steps of 16 dims with A in TMEM
-constexpr int kQtChunks = 32;      // 16-byte query chunks held in TMEM
+constexpr uint32_t kColO = 0;             // 256 columns
+constexpr uint32_t kColS = 256;           // 2 x 32 columns
+constexpr uint32_t kColQ = 320;           // 192 columns: query dims 0..383 (fp16 pairs)
+constexpr int kQtSteps = 24;              // K-steps of 16 dims with A in TMEM
 
 struct Params {
-    const uint4* q;            // bf16 [T][128][576] as 16-byte chunks (72 per head)
     const uint8_t* kv;         // [slots][576] bf16 (1152 B) or fp8 (576 B)
     const float* kv_scale;     // [slots] or nullptr
     const int* slot_table;
@@ -100,15 +109,12 @@ struct Params {
 __device__ __forceinline__ uint32_t sw128(int r, int c) {
     return (uint32_t)(r * 128 + ((c ^ (r & 7)) << 4));
 }
+
 __device__ __forceinline__ uint4 ldg16(const void* p) {
     uint4 v;
     asm volatile("ld.global.nc.v4.u32 {%0, %1, %2, %3}, [%4];"
                  : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w) : "l"(p));
     return v;
-}
-
-__device__ __forceinline__ void group_sync(int id, int threads) {
-    asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(threads) : "memory");
 }
 
 __device__ __forceinline__ uint4 lds16(uint32_t saddr) {
@@ -123,24 +129,65 @@ __device__ __forceinline__ void sts16(uint32_t saddr, uint4 v) {
                  ::"r"(saddr), "r"(v.x), "r"(v.y), "r"(v.z), "r"(v.w) : "memory");
 }
 
-// Two e4m3 codes (low byte first) -> two bf16 (exact: every e4m3 value is a bf16;
-// the hardware conversion goes through fp16, which also holds every e4m3 value).
-__device__ __forceinline__ uint32_t e4m3x2_to_bf16x2(uint32_t two) {
-    const __half2_raw h = __nv_cvt_fp8x2_to_halfraw2((__nv_fp8x2_storage_t)two, __NV_E4M3);
-    const float2 f = __half22float2(*reinterpret_cast<const __half2*>(&h));
-    const __nv_bfloat162 b = __floats2bfloat162_rn(f.x, f.y);
-    return *reinterpret_cast<const uint32_t*>(&b);
+// ---------------------------------------------------------------- pair plumbing
+// Arrives on the barrier at the same offset in the even CTA of the cluster.  The
+// arrive keeps the default release semantics at CTA scope: a cluster-scope release
+// holds the issuing thread ~1000 cycles (measured), and what the even CTA consumes
+// after the barrier is read through the async proxy (each writer has already fenced
+// its shared-memory stores to that proxy) or is TMEM ordered by tcgen05 fences.
+__device__ __forceinline__ void arrive_leader(uint64_t* bar) {
+    const uint32_t a = mapa(smem_u32(bar), 0);
+    asm volatile("mbarrier.arrive.shared::cluster.b64 _, [%0];" ::"r"(a) : "memory");
 }
 
-// 16-byte asynchronous copy global -> shared; src_bytes = 0 writes zeros.
-__device__ __forceinline__ void cp_async16(uint32_t saddr, const void* gptr, uint32_t src_bytes) {
-    asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;"
-                 ::"r"(saddr), "l"(gptr), "r"(src_bytes) : "memory");
-}
-__device__ __forceinline__ void cp_async_commit_wait_all() {
-    asm volatile("cp.async.commit_group;\n\tcp.async.wait_group 0;" ::: "memory");
+// Phase test / bounded wait with cluster-scope acquire (barriers the peer arrives on).
+__device__ __forceinline__ bool mbar_test_cl(uint64_t* bar, uint32_t parity) {
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.test_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok) : "r"(smem_u32(bar)), "r"(parity) : "memory");
+    return ok != 0;
 }
 
+__device__ __forceinline__ bool mbar_wait_cl(uint64_t* bar, uint32_t parity, int* check) {
+    const long long t0 = clock64();
+    while (!mbar_test_cl(bar, parity)) {
+        if (clock64() - t0 > kWaitLimitCycles) {
+            report(check, kCheckTimeout);
+            return false;
+        }
+    }
+    return true;
+}
+
+// Paired MMAs (issued by one thread of the even CTA): D (+)= A . B with fp16 operands,
+// A from shared memory or from TMEM.
+__device__ __forceinline__ void mma2_ss(uint32_t d, uint64_t a, uint64_t b, uint32_t idesc,
+                                        uint32_t acc) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::2.kind::f16 [%0], %1, %2, %3, p;\n\t}"
+        ::"r"(d), "l"(a), "l"(b), "r"(idesc), "r"(acc) : "memory");
+}
+__device__ __forceinline__ void mma2_ts(uint32_t d, uint32_t a, uint64_t b, uint32_t idesc,
+                                        uint32_t acc) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::2.kind::f16 [%0], [%1], %2, %3, p;\n\t}"
+        ::"r"(d), "r"(a), "l"(b), "r"(idesc), "r"(acc) : "memory");
+}
+// Arrives on `bar` in both CTAs of the pair once the paired MMAs issued so far are done.
+__device__ __forceinline__ void commit_pair(uint64_t* bar) {
+    asm volatile(
+        "{\n\t.reg .b16 m;\n\tmov.b16 m, 3;\n\t"
+        "tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.multicast::cluster.b64"
+        " [%0], m;\n\t}"
+        ::"r"(smem_u32(bar)) : "memory");
+}
+
+// ---------------------------------------------------------------- conversions
 // Two floats -> fp16x2 (lo in the low half), round to nearest, saturating at 65504.
 __device__ __forceinline__ uint32_t pack_f16(float lo, float hi) {
     uint32_t r;
@@ -148,13 +195,29 @@ __device__ __forceinline__ uint32_t pack_f16(float lo, float hi) {
     return r;
 }
 
-// Eight bf16 -> eight fp16: exact for magnitudes in [2^-14, 65504] (larger ones
-// saturate; smaller ones keep an absolute precision of 2^-24).
-__device__ __forceinline__ uint4 bf16x8_to_f16x8(uint4 a) {
-    auto cv = [](uint32_t v) {
-        return pack_f16(__uint_as_float(v << 16), __uint_as_float(v & 0xFFFF0000u));
-    };
-    return make_uint4(cv(a.x), cv(a.y), cv(a.z), cv(a.w));
+// Eight bf16 -> eight fp16 (see the head of the file).  `flag` collects bit 15 of each
+// half of (|x| bits + 0x3880): set exactly when |x| >= 65536 (the bf16 neighbour above
+// 65280), i.e. when the value lies beyond the fp16 range, or is inf / NaN.
+__device__ __forceinline__ uint32_t bf16x2_to_f16x2(uint32_t v, uint32_t& flag) {
+    flag |= ((v & 0x7FFF7FFFu) + 0x38803880u) & 0x80008000u;
+    return pack_f16(__uint_as_float(v << 16), __uint_as_float(v & 0xFFFF0000u));
+}
+__device__ __forceinline__ uint4 bf16x8_to_f16x8(uint4 a, uint32_t& flag) {
+    return make_uint4(bf16x2_to_f16x2(a.x, flag), bf16x2_to_f16x2(a.y, flag),
+                      bf16x2_to_f16x2(a.z, flag), bf16x2_to_f16x2(a.w, flag));
+}
+
+// Two e4m3 codes (low byte first) -> two fp16 (exact).
+__device__ __forceinline__ uint32_t e4m3x2_to_f16x2(uint32_t two) {
+    const __half2_raw h = __nv_cvt_fp8x2_to_halfraw2((__nv_fp8x2_storage_t)two, __NV_E4M3);
+    return (uint32_t)h.x | ((uint32_t)h.y << 16);
+}
+// 16 codes -> two 16-byte chunks of fp16.
+__device__ __forceinline__ void e4m3x16_to_f16(uint4 a, uint4& lo, uint4& hi) {
+    lo = make_uint4(e4m3x2_to_f16x2(a.x & 0xFFFF), e4m3x2_to_f16x2(a.x >> 16),
+                    e4m3x2_to_f16x2(a.y & 0xFFFF), e4m3x2_to_f16x2(a.y >> 16));
+    hi = make_uint4(e4m3x2_to_f16x2(a.z & 0xFFFF), e4m3x2_to_f16x2(a.z >> 16),
+                    e4m3x2_to_f16x2(a.w & 0xFFFF), e4m3x2_to_f16x2(a.w >> 16));
 }
 
 __device__ __forceinline__ float fast_exp2(float x) {
@@ -168,91 +231,119 @@ __device__ __forceinline__ uint32_t pack_bf16(float a, float b) {
     return *reinterpret_cast<const uint32_t*>(&v);
 }
 
+// The 64-dim region that V block b (0..3) of CTA `rank` covers: dims
+// {128r..128r+127, 256+128r..256+128r+127} = regions 2r, 2r+1, 4+2r, 5+2r.
+__device__ __forceinline__ int vblock_region(int b, int rank) {
+    return (b & 1) + 2 * rank + 4 * (b >> 1);
+}
+
 template <bool kFp8>
 __global__ void __launch_bounds__(kThreads, 1)
-mla_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const Params p) {
+mla_pair_kernel(const __grid_constant__ CUtensorMap tm_q, const Params p) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t* base = reinterpret_cast<uint8_t*>(
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     const uint32_t sb = smem_u32(base);
-    uint8_t* vflag = base + kOffFlag;
-    float* colscale = reinterpret_cast<float*>(base + kOffScale);
+    int* srow = reinterpret_cast<int*>(base + kOffSlot);
+    float* kscale = reinterpret_cast<float*>(base + kOffScale);
+    float* red = reinterpret_cast<float*>(base + kOffRed);
     uint64_t* bars = reinterpret_cast<uint64_t*>(base + kOffBar);
-    uint64_t* kvfull = bars + 0;    // [2] gather -> MMA / softmax     (192 arrivals)
-    uint64_t* kvempty = bars + 2;   // [2] PV done -> gather           (commit)
-    uint64_t* sfull = bars + 4;     // [2] S_j ready in buffer j%2     (commit)
-    uint64_t* pfull = bars + 6;     // [2] P_j (and any O rescale) ready (128)
-    uint64_t* pvdone = bars + 8;    // [2] P_j.V finished; buffer j%2 free (commit)
-    uint64_t* qfull = bars + 10;    // query in TMEM + shared memory   (128)
-    uint64_t* qload = bars + 11;    // query tiles landed (TMA bytes)
-    uint64_t* vconv = bars + 12;    // [2] V_v of stage s converted to fp16 (96)
+    uint64_t* full = bars + 0;      // [2] even CTA: stage gathered in both CTAs   (8 warps)
+    uint64_t* meta = bars + 2;      // [2] this CTA's slots / scales of the stage  (4 warps)
+    uint64_t* sfull = bars + 4;     // [2] S_j in TMEM buffer j%2                  (commit)
+    uint64_t* pfull = bars + 6;     // [2] even CTA: P_j written, O rescaled       (8 warps)
+    uint64_t* pvdone = bars + 8;    // [2] P_j.V done: P buffer j%2 free           (commit)
+    uint64_t* sempty = bars + 10;   // [2] stage free                              (commit)
+    uint64_t* qready = bars + 12;   // even CTA: queries in place in both CTAs     (8 warps)
+    uint64_t* qfree = bars + 13;    // query staging (in stage 0) consumed         (4 warps)
+    uint64_t* qload = bars + 14;    // query tiles landed (TMA bytes)
+    uint64_t* mmadone = bars + 15;  // every paired MMA finished                   (commit)
+    uint64_t* slots = bars + 16;    // [4] tile j's slots published in ring j%4    (2 warps)
+    uint64_t* redfull = bars + 20;  // [2] row-max halves of tile j%2 written       (4 warps)
+    uint64_t* lfull = bars + 22;    // the heads' partial sums written             (4 warps)
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + kNumBars);
+    int* s_skip = reinterpret_cast<int*>(tmem_slot + 1);
 
-    const int warp = threadIdx.x >> 5;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int rank = (int)cluster_ctarank();
     pdl_trigger();
-    const int vh = blockIdx.x & 1;                   // which half of the V columns
-    const int cid = blockIdx.x >> 1;
-    const int t = cid / p.nsplit, split = cid % p.nsplit;
-    const RowInfo ri = row_info(p.bv, t, threadIdx.x == 0 ? p.check : nullptr);
+    const int pair = blockIdx.x >> 1;
+    const int t = pair / p.nsplit, split = pair % p.nsplit;
+    const RowInfo ri = row_info(p.bv, t, (threadIdx.x == 0 && rank == 0) ? p.check : nullptr);
     const int i0 = split * p.chunk, i1 = min(p.k, i0 + p.chunk);
-    __shared__ int s_skip;
 
     if (threadIdx.x == 0) {
-        s_skip = timed_out_before(p.check) ? 1 : 0;
-        for (int i = 0; i < kStages; ++i) {
-            mbar_init(&kvfull[i], kGroupThreads);
-            mbar_init(&kvempty[i], 1);
-        }
         for (int i = 0; i < 2; ++i) {
+            mbar_init(&full[i], 16);
+            mbar_init(&meta[i], 2);
             mbar_init(&sfull[i], 1);
-            mbar_init(&pfull[i], 128);
+            mbar_init(&pfull[i], 8);
             mbar_init(&pvdone[i], 1);
+            mbar_init(&sempty[i], 1);
         }
-        mbar_init(qfull, 128);
+        mbar_init(qready, 8);
+        mbar_init(qfree, 4);
         mbar_init(qload, 1);
-        mbar_init(&vconv[0], kGroupThreads);
-        mbar_init(&vconv[1], kGroupThreads);
+        mbar_init(mmadone, 1);
+        for (int i = 0; i < 4; ++i) mbar_init(&slots[i], 2);
+        for (int i = 0; i < 2; ++i) mbar_init(&redfull[i], 4);
+        mbar_init(lfull, 4);
         fence_barrier_init();
-        // the query row block [128 heads][576] as nine 64-dim swizzled tiles: dims
-        // 256..575 straight into their shared-memory home, dims 0..255 into KV stage 0
-        // for the softmax threads to move into TMEM
-        if (ri.ok) {
-            prefetch_tmap(&tm_q);
-            mbar_arrive_expect_tx(qload, 9 * 16384);
-            for (int r = 0; r < 9; ++r)
-                tma_load_2d(base + (r < 4 ? kOffKV + r * 16384 : kOffQs + (r - 4) * 16384), &tm_q,
-                            64 * r, t * kHeads, qload);
+        if (rank == 0) {   // one decision for both CTAs: skip the work after a timeout
+            const int skip = timed_out_before(p.check) ? 1 : 0;
+            *s_skip = skip;
+            asm volatile("st.shared::cluster.u32 [%0], %1;"
+                         ::"r"(mapa(smem_u32(s_skip), 1)), "r"(skip) : "memory");
         }
     }
     if (warp == kMmaWarp) {
-        tmem_alloc(tmem_slot, kTmemCols);
-        tmem_relinquish();
+        asm volatile("tcgen05.alloc.cta_group::2.sync.aligned.shared::cta.b32 [%0], %1;"
+                     ::"r"(smem_u32(tmem_slot)), "r"(kTmemCols) : "memory");
+        asm volatile("tcgen05.relinquish_alloc_permit.cta_group::2.sync.aligned;" ::: "memory");
     }
     tc_fence_before();
-    __syncthreads();
+    cluster_sync();      // barriers of both CTAs initialised, skip flag delivered, TMEM held
     tc_fence_after();
     const uint32_t tmem = *tmem_slot;
-    const int n_tiles = (ri.ok && i1 > i0 && !s_skip) ? (i1 - i0 + kTile - 1) / kTile : 0;
+    const int n_tiles = (ri.ok && i1 > i0 && !*s_skip) ? (i1 - i0 + kTile - 1) / kTile : 0;
+
+    if (threadIdx.x == 0 && n_tiles > 0) {
+        // this CTA's 64 query rows as nine 64-dim swizzled tiles: dims 384..575 straight
+        // into their shared-memory home, dims 0..383 into stage 0 for the softmax threads
+        // to move into TMEM
+        prefetch_tmap(&tm_q);
+        mbar_arrive_expect_tx(qload, 9 * 8192);
+        for (int r = 0; r < 9; ++r)
+            tma_load_2d(base + (r < 6 ? kOffStage + r * 8192 : kOffQs + (r - 6) * 8192), &tm_q,
+                        64 * r, t * kHeads + 64 * rank, qload);
+    }
 
     if (warp >= kGatherWarp0 && warp < kMmaWarp) {
         // ============================================================ gather
-        // Group g (warps 4-6 or 7-9) fills KV stage g with tiles g, g+2, g+4, ...:
-        // the two groups' copies of consecutive tiles overlap.  Thread r < 64 of a
-        // group owns row r: it runs the index -> slot pipeline for the group's
-        // upcoming tiles and publishes the tile's slots in shared memory; then every
-        // warp copies whole 128-byte lines (8 lanes per line, 4 rows per instruction).
-        const int gt = threadIdx.x - kGatherWarp0 * 32;     // 0..191
-        const int grp = gt / kGroupThreads, gl = gt % kGroupThreads;
-        const int gw = gl >> 5, lane = gl & 31;
+        // All eight warps gather every tile.  Thread gt < 64 owns key gt of each tile
+        // (index -> slot pipeline, three tiles ahead) and publishes the tile's slots in a
+        // four-entry ring; every thread then issues its share of the tile's loads (whole
+        // 16-byte chunks, a warp covering 512 contiguous bytes of a row) into registers
+        // BEFORE waiting for the tile's stage to be released, so the loads' latency
+        // overlaps the compute of the two tiles in the stages; then it converts to fp16
+        // and stores into the swizzled stage: this CTA's 32 rows into the key buffer
+        // (and their V dims of this CTA's half into the V block), the peer's 32 rows'
+        // V dims of this half into the V block.  (A thread is at most two tiles ahead of
+        // the slowest gather thread -- a stage is released only after every thread has
+        // gathered into it -- so a ring entry is rewritten only after every thread has
+        // read it.)
+        const int gt = threadIdx.x - kGatherWarp0 * 32;       // 0..255
         constexpr int kRowBytes = kFp8 ? 576 : 1152;
-        int* srow = reinterpret_cast<int*>(base + kOffSlot) + grp * 64;
+        constexpr int kOwnChunks = kFp8 ? 32 * 36 : 32 * 72;   // 16-byte loads per tile
+        constexpr int kPeerChunks = kFp8 ? 32 * 16 : 32 * 32;
+        constexpr int kLoads = (kOwnChunks + kPeerChunks + 255) / 256;
+        int* ring = reinterpret_cast<int*>(base + kOffRing);
+        float* ring_sc = reinterpret_cast<float*>(base + kOffRingSc);
         const long long seq_base = (long long)ri.b * p.st_stride;
         auto fetch_idx = [&](int j) -> int {
-            const int i = i0 + j * kTile + gl;
-            return (gl < kTile && j < n_tiles && i < i1) ? __ldg(p.idx + (long long)t * p.k + i) : -1;
+            const int i = i0 + j * kTile + gt;
+            return (gt < kTile && j < n_tiles && i < i1) ? __ldg(p.idx + (long long)t * p.k + i) : -1;
         };
-        // Slot-table entry for index s, or a sentinel for a skipped entry / an index
-        // past the query position (table entries are checked separately).
         constexpr int kSkip = INT_MIN, kPastPos = INT_MIN + 1;
         auto fetch_slot = [&](int s) -> int {
             if (s < 0) return kSkip;
@@ -267,231 +358,316 @@ mla_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const Params p) {
             }
             return raw;
         };
-        // pipeline over the group's own tiles: slots of tiles j and j+2, the table
-        // entry of tile j+4 and the index of tile j+6 are in flight at tile j
+        auto fetch_scale = [&](int sl) -> float {
+            return (kFp8 && sl >= 0 && p.kv_scale) ? __ldg(p.kv_scale + sl) : 1.0f;
+        };
+        // index pipeline (threads gt < 64): the checked slot and scale of the next tile to
+        // publish, the slot of the one after, the raw table entry and the index beyond
         int sl_cur = -1, sl_next = -1, raw_n2 = kSkip, idx_n3 = -1;
+        float sc_cur = 1.0f;
         pdl_wait();                                  // the selection may come from the previous kernel
-        if (grp < n_tiles) {
-            const int x0 = fetch_idx(grp), x1 = fetch_idx(grp + 2), x2 = fetch_idx(grp + 4);
-            idx_n3 = fetch_idx(grp + 6);
+        if (n_tiles > 0 && gt < kTile) {
+            const int x0 = fetch_idx(0), x1 = fetch_idx(1), x2 = fetch_idx(2);
+            idx_n3 = fetch_idx(3);
             const int r0 = fetch_slot(x0), r1 = fetch_slot(x1);
             raw_n2 = fetch_slot(x2);
             sl_cur = check_slot(r0);
             sl_next = check_slot(r1);
+            sc_cur = fetch_scale(sl_cur);
         }
-        const int stage = grp;
-        const uint32_t st = sb + kOffKV + stage * kStageBytes;
-        if (grp == 0 && n_tiles > 0) mbar_wait_warp(qfull, 0, p.check);   // stage 0 held query tiles
-        for (int j = grp; j < n_tiles; j += kStages) {
-            if (sl_next >= 0)
-                asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;"
-                             ::"l"(p.kv + (long long)sl_next * kRowBytes), "r"(kRowBytes) : "memory");
-            if (!mbar_wait_warp(&kvempty[stage], ((j / kStages) & 1) ^ 1, p.check)) break;
-            if (gl < kTile) {
-                srow[gl] = sl_cur;
-                vflag[stage * 64 + gl] = sl_cur >= 0 ? 1 : 0;
-                colscale[stage * 64 + gl] =
-                    (kFp8 && sl_cur >= 0 && p.kv_scale) ? __ldg(p.kv_scale + sl_cur) : 1.0f;
+        uint32_t range = 0;
+        // Publishes tile j's slots in ring entry j % 4 (the next tile in order) and waits
+        // until the whole gather may read them.
+        auto publish = [&](int j) -> bool {
+            const int e = j & 3;
+            if (gt < kTile) {
+                ring[e * 64 + gt] = sl_cur;
+                ring_sc[e * 64 + gt] = sc_cur;
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&slots[e]);
+                const int nxt = check_slot(raw_n2);
+                raw_n2 = fetch_slot(idx_n3);
+                idx_n3 = fetch_idx(j + 4);
+                sl_cur = sl_next;
+                sl_next = nxt;
+                sc_cur = fetch_scale(sl_cur);
             }
-            group_sync(1 + grp, kGroupThreads);
-            if constexpr (!kFp8) {
-                // 64 rows x 9 regions of 128 bytes = 144 units of 4 rows; warp gw takes
-                // units gw, gw+3, ...; a skipped or bad row becomes zeros (score masked)
-                const int chunk = lane & 7;
-#pragma unroll 8
-                for (int u = gw; u < 144; u += 3) {
-                    const int rg = u / 9, region = u - rg * 9;
-                    const int row = 4 * rg + (lane >> 3);
-                    const int sl = srow[row];
-                    const uint8_t* src = p.kv + (long long)(sl < 0 ? 0 : sl) * 1152 + region * 128 + chunk * 16;
-                    cp_async16(st + region * 8192 + sw128(row, chunk), src, sl >= 0 ? 16u : 0u);
-                }
-            } else {
-                // 64 rows x 36 pieces of 16 e4m3 codes; thread gl takes pieces gl + 96 i
-                uint4 v[24];
+            return mbar_wait_warp(&slots[e], (j >> 2) & 1, p.check);
+        };
+        // Issues this thread's loads of tile j into v (the slot of every load first, all
+        // shared-memory reads in flight at once, then the global loads).
+        auto issue = [&](int j, uint4 (&v)[kLoads]) {
+            const uint32_t rs_s = sb + kOffRing + (j & 3) * 256;
+            int slv[kLoads];
+            int offv[kLoads];
 #pragma unroll
-                for (int i = 0; i < 24; ++i) {
-                    const int q = gl + kGroupThreads * i, row = q / 36, pc = q - row * 36;
-                    const int sl = srow[row];
-                    v[i] = sl >= 0 ? ldg16(p.kv + (long long)sl * 576 + pc * 16) : make_uint4(0, 0, 0, 0);
+            for (int i = 0; i < kLoads; ++i) {
+                const int q = gt + 256 * i;
+                int key = 0;
+                offv[i] = -1;
+                if (q < kOwnChunks) {
+                    const int row = kFp8 ? q / 36 : q / 72, c = kFp8 ? q - row * 36 : q - row * 72;
+                    key = 32 * rank + row;
+                    offv[i] = c * 16;
+                } else if (q < kOwnChunks + kPeerChunks) {
+                    const int qp = q - kOwnChunks;
+                    const int row = kFp8 ? qp >> 4 : qp >> 5, jq = kFp8 ? qp & 15 : qp & 31;
+                    const int reg = vblock_region(kFp8 ? jq >> 2 : jq >> 3, rank);
+                    key = 32 * (1 - rank) + row;
+                    offv[i] = kFp8 ? reg * 64 + (jq & 3) * 16 : reg * 128 + (jq & 7) * 16;
                 }
+                asm volatile("ld.shared.u32 %0, [%1];" : "=r"(slv[i]) : "r"(rs_s + 4 * key) : "memory");
+            }
 #pragma unroll
-                for (int i = 0; i < 24; ++i) {
-                    const int q = gl + kGroupThreads * i, row = q / 36, pc = q - row * 36;
-                    const int g = 2 * pc;                       // first of the two bf16 chunks
-                    const uint4 a = v[i];
-                    const uint4 lo = make_uint4(e4m3x2_to_bf16x2(a.x & 0xFFFF), e4m3x2_to_bf16x2(a.x >> 16),
-                                                e4m3x2_to_bf16x2(a.y & 0xFFFF), e4m3x2_to_bf16x2(a.y >> 16));
-                    const uint4 hi = make_uint4(e4m3x2_to_bf16x2(a.z & 0xFFFF), e4m3x2_to_bf16x2(a.z >> 16),
-                                                e4m3x2_to_bf16x2(a.w & 0xFFFF), e4m3x2_to_bf16x2(a.w >> 16));
-                    sts16(st + (g >> 3) * 8192 + sw128(row, g & 7), lo);
-                    sts16(st + ((g + 1) >> 3) * 8192 + sw128(row, (g + 1) & 7), hi);
+            for (int i = 0; i < kLoads; ++i) {
+                v[i] = make_uint4(0u, 0u, 0u, 0u);
+                if (offv[i] >= 0 && slv[i] >= 0)
+                    v[i] = ldg16(p.kv + (long long)slv[i] * kRowBytes + offv[i]);
+            }
+        };
+        // Waits for tile j's stage, then converts and stores v there and tells the
+        // attention (slots and scales for the softmax, the data for the MMA).
+        auto store = [&](int j, const uint4 (&v)[kLoads]) -> bool {
+            const int stage = j & 1;
+            // the stage is free once P_{j-2}.V has finished (stage 0 first holds the query
+            // tiles, until the softmax warps have moved them)
+            if (j == 0 && !mbar_wait_warp(qfree, 0, p.check)) return false;
+            if (!mbar_wait_warp(&sempty[stage], ((j >> 1) & 1) ^ 1, p.check)) return false;
+            if (gt < kTile) {      // the tile's slots and scales for the softmax
+                srow[stage * 64 + gt] = ring[(j & 3) * 64 + gt];
+                kscale[stage * 64 + gt] = ring_sc[(j & 3) * 64 + gt];
+            }
+            const uint32_t sbuf = sb + kOffStage + stage * kStageBytes;
+            const uint32_t vblk = sbuf + kSbufBytes;
+#pragma unroll
+            for (int i = 0; i < kLoads; ++i) {
+                const int q = gt + 256 * i;
+                if (q < kOwnChunks) {
+                    if constexpr (!kFp8) {
+                        const int row = q / 72, c = q - row * 72, reg = c >> 3, ch = c & 7;
+                        const uint4 f = bf16x8_to_f16x8(v[i], range);
+                        sts16(sbuf + reg * 4096 + sw128(row, ch), f);
+                        if (reg < 8 && ((reg >> 1) & 1) == rank)
+                            sts16(vblk + (((reg >> 2) << 1) | (reg & 1)) * 8192 + sw128(32 * rank + row, ch), f);
+                    } else {
+                        const int row = q / 36, c = q - row * 36, reg = c >> 2, ch = 2 * (c & 3);
+                        uint4 lo, hi;
+                        e4m3x16_to_f16(v[i], lo, hi);
+                        sts16(sbuf + reg * 4096 + sw128(row, ch), lo);
+                        sts16(sbuf + reg * 4096 + sw128(row, ch + 1), hi);
+                        if (reg < 8 && ((reg >> 1) & 1) == rank) {
+                            const uint32_t vb = vblk + (((reg >> 2) << 1) | (reg & 1)) * 8192;
+                            sts16(vb + sw128(32 * rank + row, ch), lo);
+                            sts16(vb + sw128(32 * rank + row, ch + 1), hi);
+                        }
+                    }
+                } else if (q < kOwnChunks + kPeerChunks) {
+                    const int qp = q - kOwnChunks;
+                    if constexpr (!kFp8) {
+                        const int row = qp >> 5, jq = qp & 31;
+                        sts16(vblk + (jq >> 3) * 8192 + sw128(32 * (1 - rank) + row, jq & 7),
+                              bf16x8_to_f16x8(v[i], range));
+                    } else {
+                        const int row = qp >> 4, jq = qp & 15, ch = 2 * (jq & 3);
+                        const uint32_t vb = vblk + (jq >> 2) * 8192;
+                        uint4 lo, hi;
+                        e4m3x16_to_f16(v[i], lo, hi);
+                        sts16(vb + sw128(32 * (1 - rank) + row, ch), lo);
+                        sts16(vb + sw128(32 * (1 - rank) + row, ch + 1), hi);
+                    }
                 }
             }
-            // advance the pipeline (independent loads, issued before waiting on the copies)
-            const int nxt = check_slot(raw_n2);     // loaded one round ago
-            raw_n2 = fetch_slot(idx_n3);             // index loaded one round ago
-            idx_n3 = fetch_idx(j + 8);
-            if constexpr (!kFp8) cp_async_commit_wait_all();
             fence_proxy_async_smem();
-            mbar_arrive(&kvfull[stage]);
-            // once S_j has read the bf16 rows, convert this CTA's V columns in place to
-            // fp16 for P.V (P is fp16: bf16 P keeps too few bits, see above)
-            if (!mbar_wait_warp(&sfull[stage], (j >> 1) & 1, p.check)) break;
-            tc_fence_after();
-            const uint32_t vb = st + vh * 4 * 8192;
-#pragma unroll 4
-            for (int q = gl; q < 4 * 512; q += kGroupThreads) {
-                const uint32_t a = vb + q * 16;
-                sts16(a, bf16x8_to_f16x8(lds16(a)));
+            __syncwarp();
+            if (lane == 0) {
+                arrive_leader(&full[stage]);
+                if (gt < kTile) mbar_arrive(&meta[stage]);
             }
-            fence_proxy_async_smem();
-            mbar_arrive(&vconv[stage]);
-            sl_cur = sl_next;
-            sl_next = nxt;
+            return true;
+        };
+        bool alive = n_tiles > 0;
+        uint4 va[kLoads];
+        if constexpr (kLoads <= 8) {
+            // two tiles of loads in flight: tile j+1's are issued before tile j is stored
+            uint4 vb[kLoads];
+            if (alive && (alive = publish(0))) issue(0, va);
+            for (int j = 0; alive && j < n_tiles; j += 2) {
+                if (j + 1 < n_tiles) {
+                    if (!(alive = publish(j + 1))) break;
+                    issue(j + 1, vb);
+                }
+                if (!(alive = store(j, va))) break;
+                if (j + 1 >= n_tiles) break;
+                if (j + 2 < n_tiles) {
+                    if (!(alive = publish(j + 2))) break;
+                    issue(j + 2, va);
+                }
+                if (!(alive = store(j + 1, vb))) break;
+            }
+        } else {
+            // one tile in flight (the registers of a second would not fit): tile j's loads
+            // are issued before its stage is free
+            for (int j = 0; alive && j < n_tiles; ++j) {
+                if (!(alive = publish(j))) break;
+                issue(j, va);
+                if (!(alive = store(j, va))) break;
+            }
         }
+        // the releases of the last two stages are the last commits aimed at the gather's
+        // barriers: wait for them, so that no arrival lands after this CTA has gone
+        for (int j = max(0, n_tiles - 2); alive && j < n_tiles; ++j)
+            alive = mbar_wait_warp(&sempty[j & 1], (j >> 1) & 1, p.check);
+        if (range) report(p.check, kCheckFp16Range);
     } else if (warp == kMmaWarp) {
         // ============================================================ MMA issuer
-        if (elect_one() && n_tiles > 0) {
-            bool alive = mbar_wait(qfull, 0, p.check);
+        if (rank == 0 && n_tiles > 0 && elect_one()) {
+            bool alive = mbar_wait_cl(qready, 0, p.check);
             tc_fence_after();
-            const uint32_t idesc_qk = instr_desc(1, 1, 0, 0, kTile, kHeads);   // bf16 x bf16
-            const uint32_t idesc_pv = instr_desc(0, 0, 0, 1, 256, kHeads);   // fp16 P x fp16 V
-            const uint32_t qs = sb + kOffQs;
-            // S_j = Q . KV_j^T (36 K-steps of 16: dims 0..255 with A in TMEM, the rest
-            // with A in shared memory)
-            auto issue_qk = [&](int jt) {
-                const uint32_t kva = sb + kOffKV + (jt % kStages) * kStageBytes;
-                const uint32_t sbuf = tmem + kColS + 64 * (jt & 1);
+            const uint32_t idesc_s = instr_desc(0, 0, 0, 0, kTile, kHeads);   // fp16 x fp16, N=64
+            const uint32_t idesc_v = instr_desc(0, 0, 0, 1, 256, kHeads);     // V MN-major, N=256
+            // S_j = Q . K_j^T: 36 K-steps of 16 dims, dims 0..383 with A in TMEM
+            auto issue_s = [&](int jt) {
+                const uint32_t kb = sb + kOffStage + (jt & 1) * kStageBytes;
+                const uint32_t d = tmem + kColS + 32 * (jt & 1);
 #pragma unroll
                 for (int s = 0; s < 36; ++s) {
-                    const uint64_t bdesc =
-                        smem_desc(kva + (s >> 2) * 8192 + (s & 3) * 32, 16, 1024, kLayoutSw128);
+                    const uint64_t bdesc = smem_desc(kb + (s >> 2) * 4096 + (s & 3) * 32, 16, 1024,
+                                                     kLayoutSw128);
                     if (s < kQtSteps)
-                        mma_f16_ts(sbuf, tmem + kColQ + 8 * s, bdesc, idesc_qk, s > 0 ? 1u : 0u);
+                        mma2_ts(d, tmem + kColQ + 8 * s, bdesc, idesc_s, s > 0 ? 1u : 0u);
                     else
-                        mma_f16(sbuf,
-                                smem_desc(qs + ((s - kQtSteps) >> 2) * 16384 + (s & 3) * 32, 16, 1024,
-                                          kLayoutSw128),
-                                bdesc, idesc_qk, 1u);
+                        mma2_ss(d, smem_desc(sb + kOffQs + ((s - kQtSteps) >> 2) * 8192 + (s & 3) * 32,
+                                             16, 1024, kLayoutSw128),
+                                bdesc, idesc_s, 1u);
                 }
-                mma_commit(&sfull[jt & 1]);
+                commit_pair(&sfull[jt & 1]);
             };
-            // O_v += P . V_v (fp16 operands; K = 64 tokens in four steps of 16)
+            // O += P_j . V_j: two N=256 halves of the 512 V dims, four K-steps of 16 keys
             auto issue_pv = [&](int jt) {
-                const int stage = jt % kStages;
-                const uint32_t va = sb + kOffKV + stage * kStageBytes + vh * 4 * 8192;
+                const uint32_t vb = sb + kOffStage + (jt & 1) * kStageBytes + kSbufBytes;
+                const uint32_t pa = sb + kOffP + (jt & 1) * kPBytes;
 #pragma unroll
-                for (int kk = 0; kk < 4; ++kk)
-                    mma_f16_ts(tmem + kColO, tmem + kColS + 64 * (jt & 1) + 8 * kk,
-                               smem_desc(va + kk * 2048, 8192, 1024, kLayoutSw128), idesc_pv,
-                               (jt > 0 || kk > 0) ? 1u : 0u);
-                mma_commit(&kvempty[stage]);
-                mma_commit(&pvdone[jt & 1]);
+                for (int m = 0; m < 2; ++m)
+#pragma unroll
+                    for (int kk = 0; kk < 4; ++kk)
+                        mma2_ss(tmem + kColO + 128 * m,
+                                smem_desc(pa + kk * 32, 16, 1024, kLayoutSw128),
+                                smem_desc(vb + 2 * m * 8192 + kk * 2048, 8192, 1024, kLayoutSw128),
+                                idesc_v, (jt > 0 || kk > 0) ? 1u : 0u);
+                commit_pair(&sempty[jt & 1]);
+                commit_pair(&pvdone[jt & 1]);
             };
-            // Round j issues S_j and P_{j-1}.V in whichever order their inputs arrive
-            // (P.V first when both are ready: it frees a KV stage for the gather).
-            // S_j reuses buffer j%2 once P_{j-2}.V has read the P stored there.
-            for (int j = 0; alive && j <= n_tiles; ++j) {
-                bool qk = j < n_tiles, pv = j >= 1;
-                const uint32_t kv_par = (j / kStages) & 1;
-                const long long t0 = clock64();
-                while (qk || pv) {
-                    if (pv && mbar_test(&pfull[(j - 1) & 1], ((j - 1) >> 1) & 1) &&
-                        mbar_test(&vconv[(j - 1) & 1], ((j - 1) >> 1) & 1)) {
-                        tc_fence_after();
-                        issue_pv(j - 1);
-                        pv = false;
-                    } else if (qk && mbar_test(&kvfull[j % kStages], kv_par) &&
-                               (j < 2 || mbar_test(&pvdone[j & 1], ((j - 2) >> 1) & 1))) {
-                        tc_fence_after();
-                        issue_qk(j);
-                        qk = false;
-                    } else if (clock64() - t0 > kWaitLimitCycles) {
-                        report(p.check, kCheckTimeout);
-                        alive = false;
-                        break;
-                    }
+            // S_js once tile js is gathered in both CTAs and its score buffer js%2 is free
+            // (P_{js-2}.V issued: the softmax of tile js-2 has read the buffer); P_jp.V once
+            // P_jp is written in both CTAs.  P.V goes first when both are ready: it frees
+            // a stage for the gather.
+            int js = 0, jp = 0;
+            long long t0 = clock64();
+            while (alive && jp < n_tiles) {
+                if (jp < js && mbar_test_cl(&pfull[jp & 1], (jp >> 1) & 1)) {
+                    tc_fence_after();
+                    issue_pv(jp++);
+                    t0 = clock64();
+                } else if (js < n_tiles && js < jp + 2 && mbar_test_cl(&full[js & 1], (js >> 1) & 1)) {
+                    tc_fence_after();
+                    issue_s(js++);
+                    t0 = clock64();
+                } else if (clock64() - t0 > kWaitLimitCycles) {
+                    report(p.check, kCheckTimeout);
+                    alive = false;
                 }
             }
+            commit_pair(mmadone);     // after everything issued above, finished or not
         }
+        __syncwarp();
+        if (n_tiles > 0) mbar_wait_warp(mmadone, 0, p.check);
     } else {
         // ============================================================ softmax
-        const int h = threadIdx.x;                       // head == TMEM lane
+        const int L = threadIdx.x;                    // TMEM lane
+        const int hl = L & 63, kh = L >> 6;           // head of this CTA, key half
         const uint32_t lane_base = tmem + ((uint32_t)(warp * 32) << 16);
-        {   // query row h, dims 0..255: from the staging tiles in KV stage 0 into TMEM
-            // (waited for whenever issued: no copy may still be in flight at exit)
-            if (ri.ok) mbar_wait_warp(qload, 0, p.check);
+        uint32_t range = 0;
+        bool alive = n_tiles > 0;
+        if (alive) {
+            // query row hl: dims 0..383 from the staging tiles into TMEM (fp16 pairs; both
+            // lanes of the head write the same row), dims 384..575 converted in place
+            alive = mbar_wait_warp(qload, 0, p.check);
+#pragma unroll 1
+            for (int r = 0; r < 6; ++r) {
+                uint32_t w[32];
+                const uint32_t src = sb + kOffStage + r * 8192;
 #pragma unroll
-            for (int g = 0; g < kQtChunks; g += 2) {
-                uint4 a = make_uint4(0, 0, 0, 0), b = a;
-                if (ri.ok) {
-                    const uint32_t src = sb + kOffKV + (g >> 3) * 16384;
-                    a = lds16(src + sw128(h, g & 7));
-                    b = lds16(src + sw128(h, (g + 1) & 7));
+                for (int c = 0; c < 8; ++c) {
+                    const uint4 f = bf16x8_to_f16x8(lds16(src + sw128(hl, c)), range);
+                    w[4 * c] = f.x;
+                    w[4 * c + 1] = f.y;
+                    w[4 * c + 2] = f.z;
+                    w[4 * c + 3] = f.w;
                 }
-                tmem_st8(lane_base + kColQ + 4 * g, a.x, a.y, a.z, a.w, b.x, b.y, b.z, b.w);
+                tmem_st32(lane_base + kColQ + 32 * r, w);
+            }
+#pragma unroll 4
+            for (int u = 0; u < 12; ++u) {
+                const int unit = L + 128 * u, r = unit >> 9, row = (unit >> 3) & 63, c = unit & 7;
+                const uint32_t a = sb + kOffQs + r * 8192 + sw128(row, c);
+                sts16(a, bf16x8_to_f16x8(lds16(a), range));
             }
             tmem_st_wait();
+            fence_proxy_async_smem();
             tc_fence_before();
-            mbar_arrive(qfull);                         // also: KV stage 0 may be refilled
+            __syncwarp();
+            if (lane == 0) {
+                arrive_leader(qready);
+                mbar_arrive(qfree);
+            }
         }
         float m_run = -INFINITY, l_run = 0.f;
-        bool alive = true;
         for (int j = 0; alive && j < n_tiles; ++j) {
-            const int stage = j % kStages;
-            float x[64];
-            const uint32_t sb_col = kColS + 64 * (j & 1);  // S_j, then P_j
-            {   // ---- scores of tile j
+            const int stage = j & 1;
+            float x[32];
+            {   // ---- scores of tile j: keys 32*kh .. 32*kh+31 of head hl
                 if (!mbar_wait_warp(&sfull[j & 1], (j >> 1) & 1, p.check)) { alive = false; break; }
                 tc_fence_after();
-                uint32_t a[32], c[32];
-                tmem_ld32(lane_base + sb_col, a);
-                tmem_ld32(lane_base + sb_col + 32, c);
+                uint32_t a[32];
+                tmem_ld32(lane_base + kColS + 32 * (j & 1), a);
                 tmem_ld_wait();
 #pragma unroll
-                for (int i = 0; i < 32; ++i) {
-                    x[i] = __uint_as_float(a[i]);
-                    x[32 + i] = __uint_as_float(c[i]);
-                }
+                for (int i = 0; i < 32; ++i) x[i] = __uint_as_float(a[i]);
             }
-            // ---- online softmax (base 2)
-            if (!mbar_wait_warp(&kvfull[stage], (j / kStages) & 1, p.check)) { alive = false; break; }
-            const float* cs = colscale + stage * 64;
-            {   // invalid entries (skipped or bad indices) score -inf
-                const uint4* f4 = reinterpret_cast<const uint4*>(vflag + stage * 64);
-                uint4 w[4];
-                bool all = true;
-#pragma unroll
-                for (int q = 0; q < 4; ++q) {
-                    w[q] = f4[q];
-                    all = all && w[q].x == 0x01010101u && w[q].y == 0x01010101u &&
-                          w[q].z == 0x01010101u && w[q].w == 0x01010101u;
-                }
-                if (!all) {
-#pragma unroll
-                    for (int q = 0; q < 4; ++q) {
-                        const uint32_t ws[4] = {w[q].x, w[q].y, w[q].z, w[q].w};
-#pragma unroll
-                        for (int b = 0; b < 16; ++b)
-                            if (!((ws[b >> 2] >> (8 * (b & 3))) & 1u)) x[16 * q + b] = -INFINITY;
-                    }
-                }
-            }
-            // scores in base 2: x * sc (fp8: times each row's kv scale)
+            if (!mbar_wait_warp(&meta[stage], (j >> 1) & 1, p.check)) { alive = false; break; }
+            const int* ts = srow + stage * 64 + 32 * kh;
+            const float* tsc = kscale + stage * 64 + 32 * kh;
             float sc = p.sc_log2;
-            if constexpr (kFp8) {
+            {   // invalid entries (skipped or bad indices) score -inf; fp8 rows x scale
+                const int4* s4 = reinterpret_cast<const int4*>(ts);
 #pragma unroll
-                for (int i = 0; i < 64; ++i) x[i] *= p.sc_log2 * cs[i];
-                sc = 1.0f;
+                for (int q = 0; q < 8; ++q) {
+                    const int4 v = s4[q];
+                    if (v.x < 0) x[4 * q] = -INFINITY;
+                    if (v.y < 0) x[4 * q + 1] = -INFINITY;
+                    if (v.z < 0) x[4 * q + 2] = -INFINITY;
+                    if (v.w < 0) x[4 * q + 3] = -INFINITY;
+                }
+                if constexpr (kFp8) {
+#pragma unroll
+                    for (int i = 0; i < 32; ++i) x[i] *= p.sc_log2 * tsc[i];
+                    sc = 1.0f;
+                }
             }
-            float mx[8];
+            float mx[4];
 #pragma unroll
-            for (int i = 0; i < 8; ++i)
+            for (int i = 0; i < 4; ++i)
                 mx[i] = fmaxf(fmaxf(fmaxf(x[8 * i], x[8 * i + 1]), fmaxf(x[8 * i + 2], x[8 * i + 3])),
                               fmaxf(fmaxf(x[8 * i + 4], x[8 * i + 5]), fmaxf(x[8 * i + 6], x[8 * i + 7])));
-            const float m_tile = sc * fmaxf(fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])),
-                                            fmaxf(fmaxf(mx[4], mx[5]), fmaxf(mx[6], mx[7])));
+            // the other half of the head's row max (lane L ^ 64, two warps away); the
+            // buffer of tile j is rewritten two tiles later, after every warp has
+            // published tile j+1 and so finished reading tile j
+            float* rb = red + (j & 1) * 128;
+            rb[L] = fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3]));
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&redfull[j & 1]);
+            if (!mbar_wait_warp(&redfull[j & 1], (j >> 1) & 1, p.check)) { alive = false; break; }
+            const float m_tile = sc * fmaxf(rb[L], rb[L ^ 64]);
             const float m_new = fmaxf(m_run, m_tile);
             const bool need = m_new > m_run + 8.0f;           // rescale only past 2^8 growth
             const float alpha = need ? fast_exp2(m_run - m_new) : 1.0f;
@@ -499,16 +675,28 @@ mla_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const Params p) {
             const bool warp_rescale = __any_sync(0xffffffffu, need) && j > 0;
             const float msub = m_run == -INFINITY ? 0.f : m_run;   // exp2(-inf) = +0
             float ls[4] = {0.f, 0.f, 0.f, 0.f};
-            uint32_t pk[32];
+            uint32_t pk[16];
 #pragma unroll
-            for (int i = 0; i < 64; i += 2) {
+            for (int i = 0; i < 32; i += 2) {
                 const float e0 = fast_exp2(fmaf(x[i], sc, -msub));
                 const float e1 = fast_exp2(fmaf(x[i + 1], sc, -msub));
                 ls[(i >> 1) & 3] += e0 + e1;
-                pk[i / 2] = kFp8 ? pack_f16(e0 * cs[i], e1 * cs[i + 1]) : pack_f16(e0, e1);
+                pk[i / 2] = kFp8 ? pack_f16(e0 * tsc[i], e1 * tsc[i + 1]) : pack_f16(e0, e1);
             }
             l_run = l_run * alpha + ((ls[0] + ls[1]) + (ls[2] + ls[3]));
-            // ---- O may be rescaled only once the previous PV has finished
+            // ---- P_j into P buffer j%2 once P_{j-2}.V has read it
+            if (j >= 2 && !mbar_wait_warp(&pvdone[j & 1], ((j - 2) >> 1) & 1, p.check)) {
+                alive = false;
+                break;
+            }
+            {
+                const uint32_t pb = sb + kOffP + (j & 1) * kPBytes;
+#pragma unroll
+                for (int q = 0; q < 4; ++q)
+                    sts16(pb + sw128(hl, 4 * kh + q),
+                          make_uint4(pk[4 * q], pk[4 * q + 1], pk[4 * q + 2], pk[4 * q + 3]));
+            }
+            // ---- O may be rescaled only once P_{j-1}.V has finished
             if (warp_rescale) {
                 if (!mbar_wait_warp(&pvdone[(j - 1) & 1], ((j - 1) >> 1) & 1, p.check)) { alive = false; break; }
                 tc_fence_after();
@@ -521,23 +709,33 @@ mla_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const Params p) {
                     for (int i = 0; i < 32; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * alpha);
                     tmem_st32(lane_base + kColO + cc * 32, o);
                 }
+                tmem_st_wait();
             }
-            tmem_st32(lane_base + sb_col, pk);
-            tmem_st_wait();
+            fence_proxy_async_smem();
             tc_fence_before();
-            mbar_arrive(&pfull[j & 1]);
+            __syncwarp();
+            if (lane == 0) arrive_leader(&pfull[j & 1]);
         }
-        // ---- epilogue: O_v / l and lse (after the predecessor kernel: an earlier kernel
-        // of the stream may still read the output or partial buffers)
+        // ---- epilogue: O / l and lse (after the predecessor kernel: an earlier kernel of
+        // the stream may still read the output or partial buffers)
         pdl_wait();
         const bool have = alive && n_tiles > 0 &&
                           mbar_wait_warp(&pvdone[(n_tiles - 1) & 1], ((n_tiles - 1) >> 1) & 1, p.check);
         tc_fence_after();
-        const float inv = (have && l_run > 0.f) ? 1.0f / l_run : 0.f;
-        const float lse_v = (have && l_run > 0.f) ? (m_run + log2f(l_run)) * 0.69314718055994531f
+        // the head's l is the sum of its two threads' partial sums
+        float* rl = red + 2 * 128;
+        rl[L] = l_run;
+        __syncwarp();
+        if (lane == 0) mbar_arrive(lfull);
+        const bool lsum = mbar_wait_warp(lfull, 0, p.check);
+        const float l_tot = l_run + (lsum ? rl[L ^ 64] : 0.f);
+        const float inv = (have && l_tot > 0.f) ? 1.0f / l_tot : 0.f;
+        const float lse_v = (have && l_tot > 0.f) ? (m_run + log2f(l_tot)) * 0.69314718055994531f
                                                   : -INFINITY;
+        const int head = 64 * rank + hl;
+        // this lane's O columns: c < 128 -> dim 128*kh + c, c >= 128 -> 256 + 128*kh + (c-128)
         if (p.nsplit == 1) {
-            uint4* orow = reinterpret_cast<uint4*>(p.out + ((long long)t * kHeads + h) * 512 + vh * 256);
+            __nv_bfloat16* orow = p.out + ((long long)t * kHeads + head) * 512;
 #pragma unroll 1
             for (int cc = 0; cc < 8; ++cc) {
                 uint32_t o[32];
@@ -545,20 +743,23 @@ mla_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const Params p) {
                     tmem_ld32(lane_base + kColO + cc * 32, o);
                     tmem_ld_wait();
                 }
+                uint4* dst = reinterpret_cast<uint4*>(orow + (cc >> 2) * 256 + 128 * kh + (cc & 3) * 32);
 #pragma unroll
                 for (int q4 = 0; q4 < 4; ++q4) {
-                    uint4 w;
-                    w.x = have ? pack_bf16(__uint_as_float(o[8 * q4 + 0]) * inv, __uint_as_float(o[8 * q4 + 1]) * inv) : 0u;
-                    w.y = have ? pack_bf16(__uint_as_float(o[8 * q4 + 2]) * inv, __uint_as_float(o[8 * q4 + 3]) * inv) : 0u;
-                    w.z = have ? pack_bf16(__uint_as_float(o[8 * q4 + 4]) * inv, __uint_as_float(o[8 * q4 + 5]) * inv) : 0u;
-                    w.w = have ? pack_bf16(__uint_as_float(o[8 * q4 + 6]) * inv, __uint_as_float(o[8 * q4 + 7]) * inv) : 0u;
-                    orow[cc * 4 + q4] = w;
+                    uint4 w = make_uint4(0u, 0u, 0u, 0u);
+                    if (have) {
+                        w.x = pack_bf16(__uint_as_float(o[8 * q4 + 0]) * inv, __uint_as_float(o[8 * q4 + 1]) * inv);
+                        w.y = pack_bf16(__uint_as_float(o[8 * q4 + 2]) * inv, __uint_as_float(o[8 * q4 + 3]) * inv);
+                        w.z = pack_bf16(__uint_as_float(o[8 * q4 + 4]) * inv, __uint_as_float(o[8 * q4 + 5]) * inv);
+                        w.w = pack_bf16(__uint_as_float(o[8 * q4 + 6]) * inv, __uint_as_float(o[8 * q4 + 7]) * inv);
+                    }
+                    dst[q4] = w;
                 }
             }
-            if (vh == 0 && p.lse) p.lse[(long long)t * kHeads + h] = lse_v;
+            if (kh == 0 && p.lse) p.lse[(long long)t * kHeads + head] = lse_v;
         } else {
-            const long long pb = ((long long)t * p.nsplit + split) * kHeads + h;
-            uint4* orow = reinterpret_cast<uint4*>(p.o_part + pb * 512 + vh * 256);
+            const long long pbase = ((long long)t * p.nsplit + split) * kHeads + head;
+            __half* orow = p.o_part + pbase * 512;
 #pragma unroll 1
             for (int cc = 0; cc < 8; ++cc) {
                 uint32_t o[32];
@@ -566,26 +767,30 @@ mla_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const Params p) {
                     tmem_ld32(lane_base + kColO + cc * 32, o);
                     tmem_ld_wait();
                 }
+                uint4* dst = reinterpret_cast<uint4*>(orow + (cc >> 2) * 256 + 128 * kh + (cc & 3) * 32);
 #pragma unroll
-                for (int q8 = 0; q8 < 4; ++q8) {
+                for (int q4 = 0; q4 < 4; ++q4) {
                     uint4 w = make_uint4(0u, 0u, 0u, 0u);
                     if (have) {
-                        w.x = pack_f16(__uint_as_float(o[8 * q8 + 0]) * inv, __uint_as_float(o[8 * q8 + 1]) * inv);
-                        w.y = pack_f16(__uint_as_float(o[8 * q8 + 2]) * inv, __uint_as_float(o[8 * q8 + 3]) * inv);
-                        w.z = pack_f16(__uint_as_float(o[8 * q8 + 4]) * inv, __uint_as_float(o[8 * q8 + 5]) * inv);
-                        w.w = pack_f16(__uint_as_float(o[8 * q8 + 6]) * inv, __uint_as_float(o[8 * q8 + 7]) * inv);
+                        w.x = pack_f16(__uint_as_float(o[8 * q4 + 0]) * inv, __uint_as_float(o[8 * q4 + 1]) * inv);
+                        w.y = pack_f16(__uint_as_float(o[8 * q4 + 2]) * inv, __uint_as_float(o[8 * q4 + 3]) * inv);
+                        w.z = pack_f16(__uint_as_float(o[8 * q4 + 4]) * inv, __uint_as_float(o[8 * q4 + 5]) * inv);
+                        w.w = pack_f16(__uint_as_float(o[8 * q4 + 6]) * inv, __uint_as_float(o[8 * q4 + 7]) * inv);
                     }
-                    orow[cc * 4 + q8] = w;
+                    dst[q4] = w;
                 }
             }
-            if (vh == 0) p.lse_part[pb] = lse_v;
+            if (kh == 0) p.lse_part[pbase] = lse_v;
         }
+        if (range) report(p.check, kCheckFp16Range);
     }
 
     tc_fence_before();
-    __syncthreads();
+    cluster_sync();          // neither CTA leaves while the pair's MMAs or arrivals may touch it
     tc_fence_after();
-    if (warp == kMmaWarp) tmem_dealloc(tmem, kTmemCols);
+    if (warp == kMmaWarp)
+        asm volatile("tcgen05.dealloc.cta_group::2.sync.aligned.b32 %0, %1;"
+                     ::"r"(tmem), "r"(kTmemCols) : "memory");
 }
 
 }  // namespace
@@ -594,7 +799,6 @@ cudaError_t launch_mla_tc(const void* q, float scale, const CacheView& kv, const
                           const int* idx, int k, int nsplit, void* out, float* lse, void* o_part,
                           float* lse_part, int* check, cudaStream_t st, bool pdl) {
     Params p;
-    p.q = reinterpret_cast<const uint4*>(q);
     p.kv = reinterpret_cast<const uint8_t*>(kv.data);
     p.kv_scale = kv.scale;
     p.slot_table = kv.table;
@@ -613,16 +817,29 @@ cudaError_t launch_mla_tc(const void* q, float scale, const CacheView& kv, const
     p.check = check;
     CUtensorMap tm_q;
     cudaError_t me = make_tensor_map_2d(&tm_q, q, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, 576,
-                                        (unsigned long long)bv.total_q * kHeads, 1152, 64, kHeads,
+                                        (unsigned long long)bv.total_q * kHeads, 1152, 64, 64,
                                         CU_TENSOR_MAP_SWIZZLE_128B);
     if (me != cudaSuccess) return me;
     const bool fp8 = kv.dtype == kE4M3;
-    auto kern = fp8 ? mla_tc_kernel<true> : mla_tc_kernel<false>;
+    auto kern = fp8 ? mla_pair_kernel<true> : mla_pair_kernel<false>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          (int)kSmemBytes);
     if (e != cudaSuccess) return e;
-    dim3 grid(2 * bv.total_q * nsplit);
-    e = launch_kernel(kern, grid, dim3(kThreads), kSmemBytes, st, pdl, tm_q, p);
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(2 * bv.total_q * nsplit);
+    cfg.blockDim = dim3(kThreads);
+    cfg.dynamicSmemBytes = kSmemBytes;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[2];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = 2;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[1].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = pdl ? 2 : 1;
+    e = cudaLaunchKernelEx(&cfg, kern, tm_q, p);
     if (e != cudaSuccess) return e;
     return cudaGetLastError();
 }
