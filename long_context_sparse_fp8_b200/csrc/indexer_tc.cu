@@ -92,6 +92,12 @@ __device__ __forceinline__ bool get_run(const Params& p, int k, Run* out, bool s
     return false;
 }
 
+// acc += a * b on a pair of floats with one packed instruction (two IEEE fp32 FMAs,
+// each rounded as fmaf would).
+__device__ __forceinline__ void ffma2(float2& acc, float2 a, float2 b) {
+    acc = __ffma2_rn(a, b, acc);
+}
+
 template <int EPI>
 __global__ void __launch_bounds__(threads_for<EPI>(), EPI == 1 ? 2 : 1)
 indexer_fp8_tc_kernel(const __grid_constant__ CUtensorMap tm_k,
@@ -259,8 +265,8 @@ indexer_fp8_tc_kernel(const __grid_constant__ CUtensorMap tm_k,
         // ------------------------------------------------------------ epilogue
         const int quarter = warp & 3;                 // TMEM lane quarter this warp may access
         const int row = quarter * 32 + lane;          // key row within the tile
-        const int q_lo = EPI == 2 ? 2 * ((warp - 2) >> 2) : 0;   // query rows of this warp
-        constexpr int kRows = EPI == 2 ? 2 : 4;
+        constexpr int kRows = EPI == 1 ? 4 : 4 / EPI;                 // query rows of this warp:
+        const int q_lo = EPI == 1 ? 0 : kRows * ((warp - 2) >> 2);     // q_lo .. q_lo + kRows - 1
         int it = 0;
         bool alive = true;
         Run run;
@@ -299,32 +305,50 @@ indexer_fp8_tc_kernel(const __grid_constant__ CUtensorMap tm_k,
                 tc_fence_after();
                 float res[4] = {0.f, 0.f, 0.f, 0.f};
                 const uint32_t tbase = tmem_base + ((uint32_t)(quarter * 32) << 16) + buf * ncols_buf;
+                // the warp's rows two at a time: all four 32-head TMEM loads are issued
+                // before one wait (a TMEM load takes a few hundred cycles; issued one
+                // after another they would serialise that latency four times)
 #pragma unroll
-                for (int u = 0; u < kRows; ++u) {
-                    const int qi = q_lo + u;
-                    if (qi >= run.r) break;
-                    uint32_t v0[32], v1[32];
-                    tmem_ld32(tbase + qi * kHeads, v0);
-                    tmem_ld32(tbase + qi * kHeads + 32, v1);
-                    tmem_ld_wait();
-                    // sum_h w_h * ReLU(D_h) in 8 independent partial sums (a single
-                    // chain of 64 dependent FMAs would dominate the tile's time)
-                    const float4* w4 = reinterpret_cast<const float4*>(w_run + qi * kHeads);
-                    float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+                for (int u0 = 0; u0 < kRows; u0 += 2) {
+                    const int nr = min(min(2, kRows - u0), run.r - (q_lo + u0));   // rows of this pair
+                    if (nr <= 0) break;
+                    uint32_t v[2][64];
 #pragma unroll
-                    for (int h4 = 0; h4 < 8; ++h4) {
-                        const float4 wa = w4[h4], wb = w4[8 + h4];
-                        const int e = (h4 & 1) * 4;
-                        acc[e + 0] = fmaf(wa.x, fmaxf(__uint_as_float(v0[4 * h4 + 0]), 0.f), acc[e + 0]);
-                        acc[e + 1] = fmaf(wa.y, fmaxf(__uint_as_float(v0[4 * h4 + 1]), 0.f), acc[e + 1]);
-                        acc[e + 2] = fmaf(wa.z, fmaxf(__uint_as_float(v0[4 * h4 + 2]), 0.f), acc[e + 2]);
-                        acc[e + 3] = fmaf(wa.w, fmaxf(__uint_as_float(v0[4 * h4 + 3]), 0.f), acc[e + 3]);
-                        acc[e + 0] = fmaf(wb.x, fmaxf(__uint_as_float(v1[4 * h4 + 0]), 0.f), acc[e + 0]);
-                        acc[e + 1] = fmaf(wb.y, fmaxf(__uint_as_float(v1[4 * h4 + 1]), 0.f), acc[e + 1]);
-                        acc[e + 2] = fmaf(wb.z, fmaxf(__uint_as_float(v1[4 * h4 + 2]), 0.f), acc[e + 2]);
-                        acc[e + 3] = fmaf(wb.w, fmaxf(__uint_as_float(v1[4 * h4 + 3]), 0.f), acc[e + 3]);
+                    for (int u = 0; u < 2; ++u) {
+                        if (u < nr) {
+                            const uint32_t c0 = tbase + (q_lo + u0 + u) * kHeads;
+                            tmem_ld32(c0, *reinterpret_cast<uint32_t(*)[32]>(&v[u][0]));
+                            tmem_ld32(c0 + 32, *reinterpret_cast<uint32_t(*)[32]>(&v[u][32]));
+                        }
                     }
-                    res[u] = ((acc[0] + acc[4]) + (acc[1] + acc[5])) + ((acc[2] + acc[6]) + (acc[3] + acc[7]));
+                    tmem_ld_wait();
+#pragma unroll
+                    for (int u = 0; u < 2; ++u) {
+                        if (u >= nr) break;
+                        const int qi = q_lo + u0 + u;
+                        // sum_h w_h * ReLU(D_h): ReLU per head, then packed pairs of FMAs
+                        // into four pair accumulators (eight independent partial sums)
+                        const uint32_t w_sa = smem_u32(w_run + qi * kHeads);
+                        float2 acc[4] = {{0.f, 0.f}, {0.f, 0.f}, {0.f, 0.f}, {0.f, 0.f}};
+#pragma unroll
+                        for (int h4 = 0; h4 < 16; ++h4) {
+                            // volatile: executed only where control reaches it (a
+                            // speculated load of a row this CTA does not have would
+                            // read past its shared memory)
+                            float4 wv;
+                            asm volatile("ld.shared.v4.f32 {%0, %1, %2, %3}, [%4];"
+                                         : "=f"(wv.x), "=f"(wv.y), "=f"(wv.z), "=f"(wv.w)
+                                         : "r"(w_sa + 16 * h4));
+                            const float2 r0 = make_float2(fmaxf(__uint_as_float(v[u][4 * h4 + 0]), 0.f),
+                                                          fmaxf(__uint_as_float(v[u][4 * h4 + 1]), 0.f));
+                            const float2 r1 = make_float2(fmaxf(__uint_as_float(v[u][4 * h4 + 2]), 0.f),
+                                                          fmaxf(__uint_as_float(v[u][4 * h4 + 3]), 0.f));
+                            ffma2(acc[(2 * h4) & 3], make_float2(wv.x, wv.y), r0);
+                            ffma2(acc[(2 * h4 + 1) & 3], make_float2(wv.z, wv.w), r1);
+                        }
+                        res[u0 + u] = ((acc[0].x + acc[0].y) + (acc[1].x + acc[1].y)) +
+                                      ((acc[2].x + acc[2].y) + (acc[3].x + acc[3].y));
+                    }
                 }
                 tc_fence_before();
                 __syncwarp();
@@ -395,11 +419,18 @@ cudaError_t launch_indexer_fp8_tc(const void* q, const float* q_scale, const flo
         e = launch_kernel(indexer_fp8_tc_kernel<1>, grid, dim3(threads_for<1>()), smem, st, pdl,
                           tm_k, tm_q, p);
         if (e != cudaSuccess) return e;
-    } else {
+    } else if (G == 3) {
         e = cudaFuncSetAttribute(indexer_fp8_tc_kernel<2>,
                                  cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
         if (e != cudaSuccess) return e;
         e = launch_kernel(indexer_fp8_tc_kernel<2>, grid, dim3(threads_for<2>()), smem, st, pdl,
+                          tm_k, tm_q, p);
+        if (e != cudaSuccess) return e;
+    } else {
+        e = cudaFuncSetAttribute(indexer_fp8_tc_kernel<4>,
+                                 cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+        if (e != cudaSuccess) return e;
+        e = launch_kernel(indexer_fp8_tc_kernel<4>, grid, dim3(threads_for<4>()), smem, st, pdl,
                           tm_k, tm_q, p);
         if (e != cudaSuccess) return e;
     }

@@ -44,6 +44,7 @@
 // softmax in base 2 with lazy rescaling (O and l are rescaled only when the running
 // max grows by more than 2^8).
 #include <climits>
+#include <type_traits>
 
 #include "kernels.h"
 #include "sm100.cuh"
@@ -394,65 +395,74 @@ mla_pair_kernel(const __grid_constant__ CUtensorMap tm_q, const Params p) {
             }
             return mbar_wait_warp(&slots[e], (j >> 2) & 1, p.check);
         };
-        // Issues this thread's loads of tile j into v (the slot of every load first, all
-        // shared-memory reads in flight at once, then the global loads).
-        auto issue = [&](int j, uint4 (&v)[kLoads]) {
+        // Issues this thread's loads I0 .. I0+N-1 of tile j into v (the slot of every load
+        // first, all shared-memory reads in flight at once, then the global loads).
+        auto issue = [&](int j, auto& v, auto i0_tag) {
+            constexpr int I0 = decltype(i0_tag)::value;
+            constexpr int N = sizeof(v) / sizeof(v[0]);
             const uint32_t rs_s = sb + kOffRing + (j & 3) * 256;
-            int slv[kLoads];
-            int offv[kLoads];
+            int slv[N];
+            int offv[N];
 #pragma unroll
-            for (int i = 0; i < kLoads; ++i) {
-                const int q = gt + 256 * i;
+            for (int ii = 0; ii < N; ++ii) {
+                const int q = gt + 256 * (I0 + ii);
                 int key = 0;
-                offv[i] = -1;
+                offv[ii] = -1;
                 if (q < kOwnChunks) {
                     const int row = kFp8 ? q / 36 : q / 72, c = kFp8 ? q - row * 36 : q - row * 72;
                     key = 32 * rank + row;
-                    offv[i] = c * 16;
+                    offv[ii] = c * 16;
                 } else if (q < kOwnChunks + kPeerChunks) {
                     const int qp = q - kOwnChunks;
                     const int row = kFp8 ? qp >> 4 : qp >> 5, jq = kFp8 ? qp & 15 : qp & 31;
                     const int reg = vblock_region(kFp8 ? jq >> 2 : jq >> 3, rank);
                     key = 32 * (1 - rank) + row;
-                    offv[i] = kFp8 ? reg * 64 + (jq & 3) * 16 : reg * 128 + (jq & 7) * 16;
+                    offv[ii] = kFp8 ? reg * 64 + (jq & 3) * 16 : reg * 128 + (jq & 7) * 16;
                 }
-                asm volatile("ld.shared.u32 %0, [%1];" : "=r"(slv[i]) : "r"(rs_s + 4 * key) : "memory");
+                asm volatile("ld.shared.u32 %0, [%1];" : "=r"(slv[ii]) : "r"(rs_s + 4 * key) : "memory");
             }
 #pragma unroll
-            for (int i = 0; i < kLoads; ++i) {
-                v[i] = make_uint4(0u, 0u, 0u, 0u);
-                if (offv[i] >= 0 && slv[i] >= 0)
-                    v[i] = ldg16(p.kv + (long long)slv[i] * kRowBytes + offv[i]);
+            for (int ii = 0; ii < N; ++ii) {
+                v[ii] = make_uint4(0u, 0u, 0u, 0u);
+                if (offv[ii] >= 0 && slv[ii] >= 0)
+                    v[ii] = ldg16(p.kv + (long long)slv[ii] * kRowBytes + offv[ii]);
             }
         };
-        // Waits for tile j's stage, then converts and stores v there and tells the
-        // attention (slots and scales for the softmax, the data for the MMA).
-        auto store = [&](int j, const uint4 (&v)[kLoads]) -> bool {
+        // Waits for tile j's stage (free once P_{j-2}.V has finished; stage 0 first holds
+        // the query tiles until the softmax warps have moved them) and hands the tile's
+        // slots and scales to the softmax.
+        auto claim = [&](int j) -> bool {
             const int stage = j & 1;
-            // the stage is free once P_{j-2}.V has finished (stage 0 first holds the query
-            // tiles, until the softmax warps have moved them)
             if (j == 0 && !mbar_wait_warp(qfree, 0, p.check)) return false;
             if (!mbar_wait_warp(&sempty[stage], ((j >> 1) & 1) ^ 1, p.check)) return false;
-            if (gt < kTile) {      // the tile's slots and scales for the softmax
+            if (gt < kTile) {
                 srow[stage * 64 + gt] = ring[(j & 3) * 64 + gt];
                 kscale[stage * 64 + gt] = ring_sc[(j & 3) * 64 + gt];
             }
-            const uint32_t sbuf = sb + kOffStage + stage * kStageBytes;
+            return true;
+        };
+        // Converts loads I0 .. I0+N-1 of tile j (in v) to fp16 and stores them into its
+        // stage: this CTA's rows into the key buffer (and their V dims of this CTA's half
+        // into the V block), the peer's rows' V dims into the V block.
+        auto put = [&](int j, const auto& v, auto i0_tag) {
+            constexpr int I0 = decltype(i0_tag)::value;
+            constexpr int N = sizeof(v) / sizeof(v[0]);
+            const uint32_t sbuf = sb + kOffStage + (j & 1) * kStageBytes;
             const uint32_t vblk = sbuf + kSbufBytes;
 #pragma unroll
-            for (int i = 0; i < kLoads; ++i) {
-                const int q = gt + 256 * i;
+            for (int ii = 0; ii < N; ++ii) {
+                const int q = gt + 256 * (I0 + ii);
                 if (q < kOwnChunks) {
                     if constexpr (!kFp8) {
                         const int row = q / 72, c = q - row * 72, reg = c >> 3, ch = c & 7;
-                        const uint4 f = bf16x8_to_f16x8(v[i], range);
+                        const uint4 f = bf16x8_to_f16x8(v[ii], range);
                         sts16(sbuf + reg * 4096 + sw128(row, ch), f);
                         if (reg < 8 && ((reg >> 1) & 1) == rank)
                             sts16(vblk + (((reg >> 2) << 1) | (reg & 1)) * 8192 + sw128(32 * rank + row, ch), f);
                     } else {
                         const int row = q / 36, c = q - row * 36, reg = c >> 2, ch = 2 * (c & 3);
                         uint4 lo, hi;
-                        e4m3x16_to_f16(v[i], lo, hi);
+                        e4m3x16_to_f16(v[ii], lo, hi);
                         sts16(sbuf + reg * 4096 + sw128(row, ch), lo);
                         sts16(sbuf + reg * 4096 + sw128(row, ch + 1), hi);
                         if (reg < 8 && ((reg >> 1) & 1) == rank) {
@@ -466,51 +476,68 @@ mla_pair_kernel(const __grid_constant__ CUtensorMap tm_q, const Params p) {
                     if constexpr (!kFp8) {
                         const int row = qp >> 5, jq = qp & 31;
                         sts16(vblk + (jq >> 3) * 8192 + sw128(32 * (1 - rank) + row, jq & 7),
-                              bf16x8_to_f16x8(v[i], range));
+                              bf16x8_to_f16x8(v[ii], range));
                     } else {
                         const int row = qp >> 4, jq = qp & 15, ch = 2 * (jq & 3);
                         const uint32_t vb = vblk + (jq >> 2) * 8192;
                         uint4 lo, hi;
-                        e4m3x16_to_f16(v[i], lo, hi);
+                        e4m3x16_to_f16(v[ii], lo, hi);
                         sts16(vb + sw128(32 * (1 - rank) + row, ch), lo);
                         sts16(vb + sw128(32 * (1 - rank) + row, ch + 1), hi);
                     }
                 }
             }
+        };
+        // Tile j is in its stage: tell the MMA issuer (both CTAs) and the softmax.
+        auto done = [&](int j) {
             fence_proxy_async_smem();
             __syncwarp();
             if (lane == 0) {
-                arrive_leader(&full[stage]);
-                if (gt < kTile) mbar_arrive(&meta[stage]);
+                arrive_leader(&full[j & 1]);
+                if (gt < kTile) mbar_arrive(&meta[j & 1]);
             }
-            return true;
         };
+        using I0_0 = std::integral_constant<int, 0>;
         bool alive = n_tiles > 0;
-        uint4 va[kLoads];
-        if constexpr (kLoads <= 8) {
+        if constexpr (kFp8) {
             // two tiles of loads in flight: tile j+1's are issued before tile j is stored
-            uint4 vb[kLoads];
-            if (alive && (alive = publish(0))) issue(0, va);
+            uint4 va[kLoads], vb[kLoads];
+            if (alive && (alive = publish(0))) issue(0, va, I0_0{});
             for (int j = 0; alive && j < n_tiles; j += 2) {
                 if (j + 1 < n_tiles) {
                     if (!(alive = publish(j + 1))) break;
-                    issue(j + 1, vb);
+                    issue(j + 1, vb, I0_0{});
                 }
-                if (!(alive = store(j, va))) break;
+                if (!(alive = claim(j))) break;
+                put(j, va, I0_0{});
+                done(j);
                 if (j + 1 >= n_tiles) break;
                 if (j + 2 < n_tiles) {
                     if (!(alive = publish(j + 2))) break;
-                    issue(j + 2, va);
+                    issue(j + 2, va, I0_0{});
                 }
-                if (!(alive = store(j + 1, vb))) break;
+                if (!(alive = claim(j + 1))) break;
+                put(j + 1, vb, I0_0{});
+                done(j + 1);
             }
         } else {
-            // one tile in flight (the registers of a second would not fit): tile j's loads
-            // are issued before its stage is free
+            // a tile's loads in two halves (two whole tiles would not fit in registers):
+            // the second half of tile j is in flight while the first is stored, and the
+            // first half of tile j+1 while the second is stored
+            constexpr int kA = (kLoads + 1) / 2;
+            using I0_A = std::integral_constant<int, kA>;
+            uint4 ra[kA], rb[kLoads - kA];
+            if (alive && (alive = publish(0))) issue(0, ra, I0_0{});
             for (int j = 0; alive && j < n_tiles; ++j) {
-                if (!(alive = publish(j))) break;
-                issue(j, va);
-                if (!(alive = store(j, va))) break;
+                issue(j, rb, I0_A{});
+                if (!(alive = claim(j))) break;
+                put(j, ra, I0_0{});
+                if (j + 1 < n_tiles) {
+                    if (!(alive = publish(j + 1))) break;
+                    issue(j + 1, ra, I0_0{});
+                }
+                put(j, rb, I0_A{});
+                done(j);
             }
         }
         // the releases of the last two stages are the last commits aimed at the gather's
