@@ -152,9 +152,10 @@ DSA_API dsa_status_t dsa_topk(const float* logits, int64_t ld_logits, const dsa_
  *   out      [T][heads][d_v] of out_dtype;  lse [T][heads] fp32 or NULL
  *            (natural log; -inf and o = 0 for a row with no valid index)
  * Kernels: BF16 q with BF16 or FP8 (per-token scale) KV, heads = 128,
- *          d_qk = 576, d_v = 512, out BF16 (tcgen05 tensor cores; S = q.kv^T on
- *          bf16 operands, P.V on fp16 operands, so V entries beyond +-65504
- *          saturate);
+ *          d_qk = 576, d_v = 512, out BF16 (tcgen05 tensor cores on pairs of
+ *          SMs; S = q.kv^T and P.V on fp16 operands: fp8 codes convert exactly,
+ *          bf16 q and rows within +-65504; a value fp16 cannot hold saturates and
+ *          is reported as DSA_CHECK_FP16_RANGE);
  *          F32 q/KV with heads <= 16, d_qk <= 576, d_v <= 512, d_v % 4 == 0
  *          (CUDA cores).
  */

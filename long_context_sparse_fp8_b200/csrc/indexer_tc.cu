@@ -273,10 +273,18 @@ indexer_fp8_tc_kernel(const __grid_constant__ CUtensorMap tm_k,
         for (int k = 0; alive && get_run(p, k, &run, skip); ++k) {
             if (run.j0 >= run.j1) continue;
             const float* w_run = w_s + (run.t0 - p.row0 - blockIdx.x * p.G) * kHeads;
-            float qs[4];
+            // this warp's rows of the run: logits row, query scale, position (registers,
+            // indexed by the unrolled row number)
+            float* rowp[kRows];
+            float qsc[kRows];
+            int posr[kRows];
 #pragma unroll
-            for (int i = 0; i < 4; ++i)
-                qs[i] = (i < run.r && p.q_scale) ? __ldg(p.q_scale + run.t0 + i) : 1.0f;
+            for (int u = 0; u < kRows; ++u) {
+                const int qi = q_lo + u;
+                rowp[u] = p.logits + (long long)(run.t0 + qi - p.row0) * p.ld;
+                qsc[u] = (qi < run.r && p.q_scale) ? __ldg(p.q_scale + run.t0 + qi) : 1.0f;
+                posr[u] = run.pos_lo + qi;
+            }
             const int pos_hi = run.pos_lo + run.r - 1;
             // this key's block-table entry two tiles ahead and its scale one tile ahead
             // (a table -> scale load chain per tile would stall every tile)
@@ -355,11 +363,9 @@ indexer_fp8_tc_kernel(const __grid_constant__ CUtensorMap tm_k,
                 if (lane == 0) mbar_arrive(&tempty[buf]);
 #pragma unroll
                 for (int u = 0; u < kRows; ++u) {
-                    const int qi = q_lo + u;
-                    if (qi >= run.r) break;
-                    const int pos = run.pos_lo + qi;
-                    float* dst = p.logits + (long long)(run.t0 + qi - p.row0) * p.ld + s;
-                    if (s <= pos) *dst = bad ? -INFINITY : res[u] * ks * qs[qi];
+                    if (q_lo + u >= run.r) break;
+                    float* dst = rowp[u] + s;
+                    if (s <= posr[u]) *dst = bad ? -INFINITY : res[u] * ks * qsc[u];
                     else if (s < p.ld) *dst = -INFINITY;
                 }
             }

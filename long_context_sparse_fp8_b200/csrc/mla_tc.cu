@@ -58,7 +58,6 @@ constexpr int kHeads = 128;
 constexpr int kTile = 64;                 // keys per tile (32 per CTA)
 constexpr int kThreads = 416;
 constexpr int kGatherWarp0 = 4;
-constexpr int kGroupThreads = 128;
 constexpr int kMmaWarp = 12;
 constexpr int kStages = 2;
 

@@ -384,13 +384,14 @@ def test_back_to_back_fused_decodes_share_a_workspace():
             assert torch.equal(r_lse, g_lse), rep
 
 
-@pytest.mark.parametrize("where", ["kv", "q"])
+@pytest.mark.parametrize("where", ["kv", "q", "q_fp8_cache"])
 def test_fp16_range_is_reported(where):
     """The tensor-core attention computes on fp16 operands: a bf16 latent-KV row or query
-    with entries beyond +-65504 cannot be represented there, and the call must say so
-    (DSA_CHECK_FP16_RANGE) instead of returning silently saturated results.  Rows of
-    ordinary magnitude in the same call are still exact."""
-    spec = W.Spec(name="range", seq_lens=[3000, 2500], nq=[3, 2], topk=2048, seed=91)
+    (next to a bf16 or an fp8 cache) with entries beyond +-65504 cannot be represented
+    there, and the call must say so (DSA_CHECK_FP16_RANGE) instead of returning silently
+    saturated results.  Rows of ordinary magnitude in the same call are still exact."""
+    spec = W.Spec(name="range", seq_lens=[3000, 2500], nq=[3, 2], topk=2048,
+                  kv_fp8=(where == "q_fp8_cache"), seed=91)
     wl = W.make(spec, device="cuda")
     if where == "kv":
         wl.kv[17, :8] = 1.0e5                      # slot 17 = position 17 of sequence 0
