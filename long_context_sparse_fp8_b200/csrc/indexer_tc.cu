@@ -16,8 +16,8 @@
 // of 128-byte-swizzled tiles), warp 1 allocates TMEM and issues the MMAs (double-
 // buffered accumulators), the epilogue warps drain TMEM and write the logits: one
 // warpgroup for one or two query rows per CTA (2 CTAs per SM), two warpgroups for
-// three or four rows (1 CTA per SM: the accumulators fill TMEM; each warpgroup
-// reduces two rows).
+// three rows and four for four (1 CTA per SM: the accumulators fill TMEM).  With four,
+// each accumulator buffer has its own two warpgroups of two rows each, a tile apart.
 //
 // Grid: x = groups of G consecutive query rows (G = 1 for one query per sequence,
 // 2 or 3 for multi-token decode, 4 otherwise; a group that spans sequences is
@@ -43,6 +43,12 @@ constexpr int kRowBytes = kHeads * kDim;            // one query row: 8 KB
 // reduces two of the rows of every tile).
 template <int EPI>
 constexpr int threads_for() { return 64 + 128 * EPI; }
+// With four epilogue warpgroups, warpgroups 0-1 reduce the even tiles (accumulator
+// buffer 0) and 2-3 the odd ones, two rows each: the two halves then work a tile apart,
+// so one half's waits and loads overlap the other half's arithmetic (all four on every
+// tile, one row each, move in lockstep and leave the SM's ALUs idle half the time).
+template <int EPI>
+constexpr int kEpiWarpsPerBuf = EPI == 4 ? 8 : 4 * EPI;
 
 struct Params {
     const float* w;
@@ -132,7 +138,7 @@ indexer_fp8_tc_kernel(const __grid_constant__ CUtensorMap tm_k,
         }
         for (int i = 0; i < 2; ++i) {
             mbar_init(&tfull[i], 1);
-            mbar_init(&tempty[i], 4 * EPI);   // one arrive per epilogue warp
+            mbar_init(&tempty[i], kEpiWarpsPerBuf<EPI>);   // one arrive per warp that reads it
         }
         mbar_init(qfull, 1);
         mbar_init(qempty, 1);
@@ -265,13 +271,22 @@ indexer_fp8_tc_kernel(const __grid_constant__ CUtensorMap tm_k,
         // ------------------------------------------------------------ epilogue
         const int quarter = warp & 3;                 // TMEM lane quarter this warp may access
         const int row = quarter * 32 + lane;          // key row within the tile
-        constexpr int kRows = EPI == 1 ? 4 : 4 / EPI;                 // query rows of this warp:
-        const int q_lo = EPI == 1 ? 0 : kRows * ((warp - 2) >> 2);     // q_lo .. q_lo + kRows - 1
+        const int wg = (warp - 2) >> 2;               // epilogue warpgroup
+        constexpr int kRows = EPI == 1 ? 4 : 2;       // query rows of this warp:
+        const int q_lo = EPI == 1 ? 0 : EPI == 2 ? 2 * wg : 2 * (wg & 1);   // q_lo .. q_lo + kRows - 1
+        // tiles this warp reduces: all, or (four warpgroups) those of its buffer parity
+        constexpr int kStep = EPI == 4 ? 2 : 1;
+        const int parity = EPI == 4 ? wg >> 1 : 0;
+        // rows whose TMEM loads are issued before one wait (EPI = 4 has no registers for two)
+        constexpr int kPair = EPI == 4 ? 1 : 2;
         int it = 0;
         bool alive = true;
         Run run;
         for (int k = 0; alive && get_run(p, k, &run, skip); ++k) {
             if (run.j0 >= run.j1) continue;
+            const int it0 = it;
+            it += run.j1 - run.j0;
+            const int jf = run.j0 + (kStep == 2 ? ((parity - it0) & 1) : 0);   // first tile of this warp
             const float* w_run = w_s + (run.t0 - p.row0 - blockIdx.x * p.G) * kHeads;
             // this warp's rows of the run: logits row, query scale, position (registers,
             // indexed by the unrolled row number)
@@ -298,31 +313,34 @@ indexer_fp8_tc_kernel(const __grid_constant__ CUtensorMap tm_k,
                 if (jt >= run.j1 || sk > pos_hi || pg < 0 || (long long)pg >= p.num_pages) return 0.f;
                 return p.k_scale ? __ldg(p.k_scale + (long long)pg * 64 + (sk & 63)) : 1.0f;
             };
-            int pg1 = tbl(run.j0), pg2 = tbl(run.j0 + 1);
-            float ks1 = scl(run.j0, pg1);
-            for (int j = run.j0; j < run.j1; ++j, ++it) {
-                const int buf = it & 1;
+            int pg1 = tbl(jf), pg2 = tbl(jf + kStep);
+            float ks1 = scl(jf, pg1);
+            for (int j = jf; j < run.j1; j += kStep) {
+                const int itj = it0 + (j - run.j0);
+                const int buf = itj & 1;
                 const int s = j * kTileKeys + row;
                 const int page = pg1;
                 const float ks = ks1;
                 const int bad = (s <= pos_hi && (page < 0 || (long long)page >= p.num_pages)) ? 1 : 0;
                 pg1 = pg2;
-                pg2 = tbl(j + 2);
-                ks1 = scl(j + 1, pg1);
-                if (!mbar_wait_warp(&tfull[buf], (it >> 1) & 1, p.check)) { alive = false; break; }
+                pg2 = tbl(j + 2 * kStep);
+                ks1 = scl(j + kStep, pg1);
+                if (!mbar_wait_warp(&tfull[buf], (itj >> 1) & 1, p.check)) { alive = false; break; }
                 tc_fence_after();
-                float res[4] = {0.f, 0.f, 0.f, 0.f};
+                float res[kRows];
+#pragma unroll
+                for (int u = 0; u < kRows; ++u) res[u] = 0.f;
                 const uint32_t tbase = tmem_base + ((uint32_t)(quarter * 32) << 16) + buf * ncols_buf;
-                // the warp's rows two at a time: all four 32-head TMEM loads are issued
-                // before one wait (a TMEM load takes a few hundred cycles; issued one
-                // after another they would serialise that latency four times)
+                // the warp's rows kPair at a time: all their 32-head TMEM loads are issued
+                // before one wait (a TMEM load takes a few hundred cycles; issued one after
+                // another they would serialise that latency)
 #pragma unroll
-                for (int u0 = 0; u0 < kRows; u0 += 2) {
-                    const int nr = min(min(2, kRows - u0), run.r - (q_lo + u0));   // rows of this pair
+                for (int u0 = 0; u0 < kRows; u0 += kPair) {
+                    const int nr = min(min(kPair, kRows - u0), run.r - (q_lo + u0));   // rows of this group
                     if (nr <= 0) break;
-                    uint32_t v[2][64];
+                    uint32_t v[kPair][64];
 #pragma unroll
-                    for (int u = 0; u < 2; ++u) {
+                    for (int u = 0; u < kPair; ++u) {
                         if (u < nr) {
                             const uint32_t c0 = tbase + (q_lo + u0 + u) * kHeads;
                             tmem_ld32(c0, *reinterpret_cast<uint32_t(*)[32]>(&v[u][0]));
@@ -331,7 +349,7 @@ indexer_fp8_tc_kernel(const __grid_constant__ CUtensorMap tm_k,
                     }
                     tmem_ld_wait();
 #pragma unroll
-                    for (int u = 0; u < 2; ++u) {
+                    for (int u = 0; u < kPair; ++u) {
                         if (u >= nr) break;
                         const int qi = q_lo + u0 + u;
                         // sum_h w_h * ReLU(D_h): ReLU per head, then packed pairs of FMAs
