@@ -331,12 +331,22 @@ indexer_fp8_tc_kernel(const __grid_constant__ CUtensorMap tm_k,
 #pragma unroll
                 for (int u = 0; u < kRows; ++u) res[u] = 0.f;
                 const uint32_t tbase = tmem_base + ((uint32_t)(quarter * 32) << 16) + buf * ncols_buf;
+                // the accumulator buffer is handed back to the MMA as soon as this warp's last
+                // TMEM load of the tile has completed: the arithmetic on those values then
+                // overlaps the next MMA into the buffer
+                const int my_rows = max(0, min(kRows, run.r - q_lo));
+                auto release = [&]() {
+                    tc_fence_before();
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive(&tempty[buf]);
+                };
+                if (my_rows == 0) release();
                 // the warp's rows kPair at a time: all their 32-head TMEM loads are issued
                 // before one wait (a TMEM load takes a few hundred cycles; issued one after
                 // another they would serialise that latency)
 #pragma unroll
                 for (int u0 = 0; u0 < kRows; u0 += kPair) {
-                    const int nr = min(min(kPair, kRows - u0), run.r - (q_lo + u0));   // rows of this group
+                    const int nr = min(kPair, my_rows - u0);   // rows of this group
                     if (nr <= 0) break;
                     uint32_t v[kPair][64];
 #pragma unroll
@@ -348,6 +358,7 @@ indexer_fp8_tc_kernel(const __grid_constant__ CUtensorMap tm_k,
                         }
                     }
                     tmem_ld_wait();
+                    if (u0 + kPair >= my_rows) release();
 #pragma unroll
                     for (int u = 0; u < kPair; ++u) {
                         if (u >= nr) break;
@@ -376,9 +387,6 @@ indexer_fp8_tc_kernel(const __grid_constant__ CUtensorMap tm_k,
                                       ((acc[2].x + acc[2].y) + (acc[3].x + acc[3].y));
                     }
                 }
-                tc_fence_before();
-                __syncwarp();
-                if (lane == 0) mbar_arrive(&tempty[buf]);
 #pragma unroll
                 for (int u = 0; u < kRows; ++u) {
                     if (q_lo + u >= run.r) break;
