@@ -22,7 +22,15 @@
 //   4. A block scan over the bitmap's popcounts turns it into the ascending list.
 // If C would overflow (thousands of keys in one bin, e.g. equal scores, or more than
 // a segment's worth in one warp's share), steps 2-3 fall back to radix passes over
-// the whole row and one marking sweep.  Rows longer
+// the whole row and one marking sweep.
+// Rows of at least 24k keys first try a sampled threshold (step 0): the m-th largest of
+// 2048 evenly spaced keys (low 10 bits cleared), m chosen so that about 2k keys of the row are expected at or
+// above it; one coalesced read of the row then gathers those keys (and positions) as
+// the candidates, and the exact selection runs on them as in step 3 with full 32-bit
+// keys.  The candidates hold the whole top k whenever at least k keys reach the
+// threshold, which is checked; otherwise (or on overflow) steps 1-4 run as above, so
+// the result is the same either way -- only the reads differ (one pass over the row,
+// no per-key shared-memory atomics).  Rows longer
 // than the bitmap capacity use a second kernel that refines over the whole row and
 // emits in two ordered sweeps.  Batches of a few dozen long rows (>= 32768 keys)
 // split every row over a thread-block cluster (topk_cluster_kernel, below).
@@ -43,6 +51,8 @@ constexpr int kCandCap = 8192;             // candidates: low 21 key bits + posi
 constexpr int kSeg = kCandCap / 32;        // per-warp candidate segment
 constexpr int kMaxWords = 8192;            // bitmap words: rows up to 262144 keys
 constexpr int kSmemLimit = 232448;
+constexpr int kSample = 2048;              // keys sampled for the step-0 threshold
+constexpr int kPrefilterRatio = 24;       // step 0 for rows of at least 24k keys
 constexpr int kStaticReserve = 1024;
 
 // Monotone map float -> uint32 (larger float, larger key); -0.0 maps like +0.0.
@@ -201,6 +211,34 @@ __device__ __forceinline__ void stage_and_histogram(const float* grow, int n, ui
     }
 }
 
+// The `need` lowest positions among the keys equal to the threshold (eqmap, n_eq of
+// them) join the selection bitmap.  Ends synchronised.
+__device__ __forceinline__ void take_lowest_equal(Shared& sh, uint32_t* bitmap, const uint32_t* eqmap,
+                                                  int words, int need, int n_eq) {
+    const int tid = threadIdx.x;
+    if (n_eq == need) {
+        for (int w = tid; w < words; w += kThreads) bitmap[w] |= eqmap[w];
+    } else {
+        const int wpt = (words + kThreads - 1) / kThreads;
+        const int w0 = min(words, tid * wpt), w1 = min(words, w0 + wpt);
+        int c = 0;
+        for (int w = w0; w < w1; ++w) c += __popc(eqmap[w]);
+        int total;
+        int before = block_excl_scan(c, sh, &total);
+        for (int w = w0; w < w1 && before < need; ++w) {
+            uint32_t e = eqmap[w];
+            const int pc = __popc(e);
+            if (before + pc > need) {               // keep only the lowest bits
+                for (int drop = before + pc - need; drop > 0; --drop)
+                    e &= ~(0x80000000u >> __clz(e));
+            }
+            bitmap[w] |= e;
+            before += pc;
+        }
+    }
+    __syncthreads();
+}
+
 // Bitmap of the selected positions (ascending) -> out[0, count).
 __device__ __forceinline__ void bitmap_to_list(Shared& sh, const uint32_t* bits, int words,
                                                int* out, int base = 0) {
@@ -252,6 +290,100 @@ topk_kernel(const float* __restrict__ logits, long long ld, BatchView bv, int k,
     const float* grow = logits + (long long)(t - row0) * ld;
     const Row row{grow, skeys, stage_cap};
     const int words = (n + 31) >> 5;
+
+    // ---- 0. sampled threshold; candidates at or above it --------------------------
+    if (n >= kPrefilterRatio * k && 3 * k <= kCandCap) {
+        uint32_t* samp = reinterpret_cast<uint32_t*>(cpos);      // [kSample], before C is built
+        for (int s = tid; s < kSample; s += kThreads)
+            samp[s] = order_key(__ldg(grow + (int)(((long long)s * n) / kSample)));
+        for (int w = tid; w < words; w += kThreads) {
+            bitmap[w] = 0u;
+            eqmap[w] = 0u;
+        }
+        __syncthreads();
+        // T0 = the m-th largest sample key with its low 10 bits cleared, m = ceil(2 k
+        // kSample / n): about 2k keys of the row are expected at or above it (the count
+        // is checked below)
+        const int m = (int)min((long long)kSample, (2LL * k * kSample + n - 1) / n);
+        auto samp_each = [&](auto f) {
+            for (int s2 = tid; s2 < kSample; s2 += kThreads) f(samp[s2]);
+        };
+        uint32_t prefix = 0u, pmask = 0u;
+        int rem = m, cnt;
+        refine(sh, hist, samp_each, 21, 11, prefix, pmask, rem, &cnt);
+        refine(sh, hist, samp_each, 10, 11, prefix, pmask, rem, &cnt);
+        const uint32_t T0 = prefix;
+        // one coalesced read of the row (a warp takes 128 consecutive keys at a time,
+        // interleaved over the warps): keys >= T0 with their positions into the
+        // sweeping warp's segment of C
+        int c_at = 0;
+        constexpr int kU = 4;                              // 128-key blocks in flight per warp
+        for (int b0 = 128 * warp; b0 < n; b0 += kU * 128 * kWarps) {        // warp-uniform
+            float4 f[kU];
+#pragma unroll
+            for (int u = 0; u < kU; ++u) {
+                const int i4 = b0 + u * 128 * kWarps + 4 * lane;
+                if (i4 + 3 < n) {
+                    f[u] = __ldg(reinterpret_cast<const float4*>(grow + i4));
+                } else {
+                    f[u].x = i4 < n ? __ldg(grow + i4) : 0.f;
+                    f[u].y = i4 + 1 < n ? __ldg(grow + i4 + 1) : 0.f;
+                    f[u].z = i4 + 2 < n ? __ldg(grow + i4 + 2) : 0.f;
+                    f[u].w = i4 + 3 < n ? __ldg(grow + i4 + 3) : 0.f;
+                }
+            }
+#pragma unroll
+            for (int u = 0; u < kU; ++u) {
+                const int i4 = b0 + u * 128 * kWarps + 4 * lane;
+                const uint32_t kk[4] = {order_key(f[u].x), order_key(f[u].y), order_key(f[u].z),
+                                        order_key(f[u].w)};
+                bool c4[4];
+#pragma unroll
+                for (int j = 0; j < 4; ++j) c4[j] = i4 + j < n && kk[j] >= T0;
+                if (!__any_sync(0xffffffffu, c4[0] || c4[1] || c4[2] || c4[3])) continue;
+#pragma unroll
+                for (int j = 0; j < 4; ++j) {
+                    const unsigned mc = __ballot_sync(0xffffffffu, c4[j]);
+                    if (mc) {
+                        const int c = c_at + __popc(mc & ((1u << lane) - 1u));
+                        if (c4[j] && c < kSeg) {
+                            ckey[warp * kSeg + c] = kk[j];
+                            cpos[warp * kSeg + c] = i4 + j;
+                        }
+                        c_at += __popc(mc);
+                    }
+                }
+            }
+        }
+        if (lane == 0) sh.seg_n[warp] = c_at;
+        int total;
+        block_excl_scan(min(c_at, kSeg + 1) * (lane == 0 ? 1 : 0), sh, &total);
+        const bool ok = !__syncthreads_or(c_at > kSeg) && total >= k;
+        if (ok) {
+            // ---- exact threshold among the candidates (full keys); mark them --------
+            const int seg_cnt = sh.seg_n[warp];
+            auto cand_each = [&](auto f) {
+                for (int c = lane; c < seg_cnt; c += 32) f(ckey[warp * kSeg + c]);
+            };
+            uint32_t pf = 0u, pm = 0u;
+            int remaining = k, n_eq;
+            refine(sh, hist, cand_each, 21, 11, pf, pm, remaining, &n_eq);
+            refine(sh, hist, cand_each, 10, 11, pf, pm, remaining, &n_eq);
+            refine(sh, hist, cand_each, 0, 10, pf, pm, remaining, &n_eq);
+            const uint32_t T = pf;
+            for (int c = lane; c < seg_cnt; c += 32) {
+                const uint32_t key = ckey[warp * kSeg + c];
+                const int p = cpos[warp * kSeg + c];
+                if (key > T) atomicOr(&bitmap[p >> 5], 1u << (p & 31));
+                else if (key == T) atomicOr(&eqmap[p >> 5], 1u << (p & 31));
+            }
+            __syncthreads();
+            take_lowest_equal(sh, bitmap, eqmap, words, remaining, n_eq);
+            bitmap_to_list(sh, bitmap, words, out);
+            return;
+        }
+        // too few keys reached T0, or a segment overflowed: the full method below
+    }
 
     // ---- 1. stage + top-bit histogram ------------------------------------------
     for (int i = tid; i < kCopies * 2048; i += kThreads) hist[i] = 0;
@@ -352,28 +484,7 @@ topk_kernel(const float* __restrict__ logits, long long ld, BatchView bv, int k,
     }
     __syncthreads();
 
-    // ---- the need_eq = remaining lowest positions among the keys equal to T ------
-    if (n_eq == remaining) {
-        for (int w = tid; w < words; w += kThreads) bitmap[w] |= eqmap[w];
-    } else {
-        const int wpt = (words + kThreads - 1) / kThreads;
-        const int w0 = min(words, tid * wpt), w1 = min(words, w0 + wpt);
-        int c = 0;
-        for (int w = w0; w < w1; ++w) c += __popc(eqmap[w]);
-        int total;
-        int before = block_excl_scan(c, sh, &total);
-        for (int w = w0; w < w1 && before < remaining; ++w) {
-            uint32_t e = eqmap[w];
-            const int pc = __popc(e);
-            if (before + pc > remaining) {          // keep only the lowest bits
-                for (int drop = before + pc - remaining; drop > 0; --drop)
-                    e &= ~(0x80000000u >> __clz(e));
-            }
-            bitmap[w] |= e;
-            before += pc;
-        }
-    }
-    __syncthreads();
+    take_lowest_equal(sh, bitmap, eqmap, words, remaining, n_eq);
 
     // ---- 4. ascending output -------------------------------------------------------
     bitmap_to_list(sh, bitmap, words, out);

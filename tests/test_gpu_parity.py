@@ -247,6 +247,41 @@ def test_topk_candidates_concentrated_in_one_warp():
     H.check_topk(got, logits.cpu().numpy(), logits.cpu().numpy(), np.array([n - 1]), k)
 
 
+@pytest.mark.parametrize("case", ["few_reach_threshold", "one_warp_overflows", "all_reach"])
+def test_topk_sampled_threshold_falls_back(case):
+    """Rows of >= 24k keys first try a threshold taken from 2048 evenly spaced keys.  Rows
+    built against it must still get the exact selection: (a) only the sampled positions
+    hold large scores, so fewer than k keys reach the sampled threshold; (b) the keys
+    that reach it all sit in the 128-key blocks one warp reads, overflowing its
+    candidate segment; (c) every key reaches it (a constant row)."""
+    n, k = 60000, 2048
+    pos = np.arange(n)
+    g = np.random.default_rng(7)
+    row = g.standard_normal(n).astype(np.float32)
+    if case == "few_reach_threshold":
+        samp = (np.arange(2048) * n) // 2048                # the sampled positions
+        row[samp] = 100.0 + np.arange(2048, dtype=np.float32)
+    elif case == "one_warp_overflows":
+        mine = np.flatnonzero((pos // 128) % 32 == 0)[:3000]
+        row[mine] = 50.0 + g.standard_normal(len(mine)).astype(np.float32)
+    else:
+        row[:] = 0.25
+    ld = (n + 3) // 4 * 4
+    logits = torch.full((1, ld), float("nan"), device="cuda")
+    logits[0, :n] = torch.from_numpy(row).cuda()
+    batch = L.Batch(torch.tensor([0, 1], dtype=torch.int32, device="cuda"),
+                    torch.tensor([n], dtype=torch.int32, device="cuda"), 1, n)
+    idx = torch.empty(1, k, dtype=torch.int32, device="cuda")
+    L.dsa_topk(logits, batch, k, idx)
+    got = idx.cpu().numpy()
+    assert L.dsa_device_check() == 0
+    H.check_topk(got, logits.cpu().numpy(), logits.cpu().numpy(), np.array([n - 1]), k)
+    if case == "few_reach_threshold":
+        assert np.array_equal(got[0], (np.arange(2048) * n) // 2048)
+    if case == "all_reach":
+        assert np.array_equal(got[0], np.arange(k))
+
+
 @pytest.mark.parametrize("kind", ["normal", "coarse", "three"])
 def test_topk_cluster_split_matches_one_cta_per_row(kind):
     """Short batches of long rows split each row over a cluster of 8, 4 or 2 CTAs;
