@@ -245,8 +245,11 @@ DSA_API dsa_status_t dsa_decode(const void* q_idx, dsa_dtype_t q_idx_dtype,
  * block's logits go to the workspace and are selected from at once, so they do not
  * round-trip through HBM and the memory needed is one block, not [T][L].
  * Arguments and results are those of dsa_indexer_logits followed by dsa_topk
- * (idx [T][k]: identical lists); workspace: dsa_indexer_topk_workspace_size bytes,
- * 16-byte aligned, contents undefined afterwards.  Meant for prefill-sized batches;
+ * (idx [T][k]: identical lists); workspace: at least dsa_indexer_topk_workspace_size
+ * bytes, 16-byte aligned, contents undefined afterwards.  A larger workspace takes
+ * larger blocks (the whole batch if its logits fit, else 148 x 2^m rows): fewer,
+ * longer launches whose logits no longer stay in L2 -- with the whole batch in one
+ * block this is dsa_indexer_logits followed by dsa_topk.  Meant for prefill-sized batches;
  * for decode, dsa_decode keeps the whole step in one call.
  */
 DSA_API size_t dsa_indexer_topk_workspace_size(const dsa_batch_t* batch);

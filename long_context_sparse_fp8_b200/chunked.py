@@ -24,9 +24,14 @@ from .workloads import INDEXER_PAGE, ChunkedWorkload
 class ChunkedPrefill:
     """Buffers and calls of a whole chunked prefill on one GPU: the selection
     [n_chunks, chunk_q, k] int32, the outputs [n_chunks, chunk_q, heads, d_v] bf16 and
-    lse [n_chunks, chunk_q, heads] fp32, and the indexer + top-k workspace."""
+    lse [n_chunks, chunk_q, heads] fp32, and the indexer + top-k workspace.
 
-    def __init__(self, cw: ChunkedWorkload):
+    ``select_blocks="chunk"`` (the default) gives dsa_indexer_topk a workspace for a
+    whole chunk's logits (8192 x 131072 fp32 = 4.3 GB at the last chunk), so each
+    chunk's indexer and top-k run as one launch each; ``"l2"`` gives it the minimum,
+    so it works in L2-sized row blocks (about 80 MB of logits, hundreds of launches)."""
+
+    def __init__(self, cw: ChunkedWorkload, select_blocks: str = "chunk"):
         import torch
         s = cw.spec
         self.cw, self.s = cw, s
@@ -38,7 +43,11 @@ class ChunkedPrefill:
         self.idx = torch.empty(C, Q, s.topk, dtype=torch.int32, device=dev)
         self.out = torch.empty(C, Q, s.heads, s.d_v, dtype=torch.bfloat16, device=dev)
         self.lse = torch.empty(C, Q, s.heads, device=dev)
+        if select_blocks not in ("chunk", "l2"):
+            raise ValueError("select_blocks must be 'chunk' or 'l2'")
         n = max(L.dsa_indexer_topk_workspace_size(b) for b in self.batches)
+        if select_blocks == "chunk":
+            n = max(n, Q * ((Q * C + 63) // 64 * 64) * 4)
         self.ws = torch.empty(max(n, 16), dtype=torch.uint8, device=dev)
 
     def rows(self, c: int):
@@ -96,16 +105,20 @@ class ChunkedPrefill:
         """Kernel launches of one step: two stores, the indexer and top-k once per row
         block, and the attention, per chunk."""
         n = 0
+        ws = self.ws.numel()
         for b in self.batches:
             ld = (b.max_seq_len + 63) // 64 * 64
-            rows = _block_rows(b.total_q, ld)
+            rows = _block_rows(b.total_q, ld, ws)
             n += 2 + 2 * ((b.total_q + rows - 1) // rows) + 1
         return n
 
 
-def _block_rows(total_q: int, ld: int) -> int:
-    """Rows per block of dsa_indexer_topk (the library's rule, restated for counting)."""
-    budget = (80 << 20) // (ld * 4)
+def _block_rows(total_q: int, ld: int, ws_bytes: int = 0) -> int:
+    """Rows per block of dsa_indexer_topk for a workspace of ws_bytes (the library's
+    rule, restated for counting)."""
+    budget = max(80 << 20, ws_bytes) // (ld * 4)
+    if budget >= total_q:
+        return total_q
     if budget >= 148:
         rows = 148
         while rows * 2 <= budget:

@@ -465,16 +465,20 @@ DSA_API dsa_status_t dsa_decode(const void* q_idx, dsa_dtype_t q_idx_dtype,
     return e == cudaSuccess ? ok() : cuda_fail(e, "decode launch");
 }
 
-// Rows per block of dsa_indexer_topk: the logits of one block take at most 80 MB of the
-// 126 MB L2, so the top-k reads them while they are still on chip.  Where that allows
-// 148 rows or more, 148 x 2^m rows: the top-k runs one CTA per row and the indexer 4 rows
-// per CTA over 592 / (rows / 4) key chunks, so both fill whole waves of the 148 SMs.
+// Rows per block of dsa_indexer_topk for a workspace of `bytes` (by default the minimum:
+// the logits of one block take at most 80 MB of the 126 MB L2, so the top-k reads them
+// while they are still on chip).  The whole batch if it fits; else, where the workspace
+// allows 148 rows or more, 148 x 2^m rows: the top-k runs one CTA per row and the indexer
+// 4 rows per CTA over 592 / (rows / 4) key chunks, so both fill whole waves of the 148
+// SMs.
 constexpr size_t kL2BlockBytes = (size_t)80 << 20;
 
-int indexer_topk_block_rows(int total_q, long long ld) {
-    const long long budget = (long long)(kL2BlockBytes / ((size_t)ld * sizeof(float)));
+int indexer_topk_block_rows(int total_q, long long ld, size_t bytes = kL2BlockBytes) {
+    const long long budget = (long long)(bytes / ((size_t)ld * sizeof(float)));
     long long rows;
-    if (budget >= kNumSMs) {
+    if (budget >= total_q) {
+        rows = total_q;                    // the whole batch in one block
+    } else if (budget >= kNumSMs) {
         rows = kNumSMs;
         while (rows * 2 <= budget) rows *= 2;
     } else {
@@ -519,7 +523,9 @@ DSA_API dsa_status_t dsa_indexer_topk(const void* q, dsa_dtype_t q_dtype, const 
     // Blocks of rows: the indexer writes a block's logits, the top-k selects from them
     // (programmatic dependents; each kernel waits for its predecessor before touching
     // the shared buffer, so block i+1's logits never overwrite what block i still reads).
-    const int rows = indexer_topk_block_rows(bv.total_q, ld);
+    // a workspace larger than the minimum takes larger blocks (fewer, longer launches)
+    const int rows = indexer_topk_block_rows(bv.total_q, ld, workspace_bytes > kL2BlockBytes
+                                                                 ? workspace_bytes : kL2BlockBytes);
     for (int r0 = 0; e == cudaSuccess && r0 < bv.total_q; r0 += rows) {
         BatchView blk = bv;
         blk.total_q = r0 + rows < bv.total_q ? r0 + rows : bv.total_q;

@@ -320,7 +320,8 @@ def test_topk_cluster_split_matches_one_cta_per_row(kind):
 def test_indexer_topk_blocks_match_separate_calls(which):
     """dsa_indexer_topk (L2-sized row blocks, no full logits matrix) selects exactly what
     dsa_indexer_logits + dsa_topk select: 14 blocks of up to 592 rows on the 32K prefill
-    (FP8 tensor-core indexer), 4 blocks on an fp32 case (CUDA-core indexer)."""
+    (FP8 tensor-core indexer), 4 blocks on an fp32 case (CUDA-core indexer); and so it
+    does with larger workspaces (larger blocks, up to the whole batch in one)."""
     if which == "prefill_32k":
         wl = _wl("c3", W.prefill_32k)
     elif which == "ragged":
@@ -345,6 +346,17 @@ def test_indexer_topk_blocks_match_separate_calls(which):
     torch.cuda.synchronize()
     assert L.dsa_device_check() == 0
     assert torch.equal(idx, idx2)
+    # larger workspaces take larger blocks: 148 x 2^m rows, then the whole batch at once
+    for bytes_ in (2 * 148 * ld * 4 + 100, s.total_q * ld * 4):
+        if bytes_ <= ws_bytes:
+            continue
+        ws_big = torch.empty(bytes_, dtype=torch.uint8, device="cuda")
+        idx3 = torch.full_like(idx, -7)
+        L.dsa_indexer_topk(wl.q_idx, None, wl.w, kc, batch, s.topk, idx3, workspace=ws_big)
+        torch.cuda.synchronize()
+        assert L.dsa_device_check() == 0
+        assert torch.equal(idx, idx3), bytes_
+        del ws_big
     rows = H.sample_rows(s.total_q, 6, seed=41)
     pos = H.positions(wl)[rows]
     g = logits.cpu().numpy()[rows]
