@@ -223,8 +223,16 @@ indexer_fp8_tc_kernel(const __grid_constant__ CUtensorMap tm_k,
                     load_pages(j4 + 8, nxt);
                 }
             }
-            // drain: every issued stage has been consumed (its empty phase completed)
+            // drain: every issued copy has landed (full phase; also after a timeout, so
+            // that no TMA write into this CTA's shared memory is in flight when it exits)
+            // and, on the normal path, every stage has been consumed (empty phase)
             const int n = it < kStages ? it : kStages;
+            bool landed = true;
+            for (int i = 0; i < n && landed; ++i) {
+                const int itx = it - 1 - i;
+                landed = mbar_wait(&full[itx % kStages], (itx / kStages) & 1, p.check);
+            }
+            if (runs_issued > 0 && landed) mbar_wait(qfull, (runs_issued - 1) & 1, p.check);
             for (int i = 0; i < n && alive; ++i) {
                 const int itx = it - 1 - i;
                 if (!mbar_wait(&empty[itx % kStages], (itx / kStages) & 1, p.check)) break;
