@@ -650,6 +650,32 @@ mla_pair_kernel(const __grid_constant__ CUtensorMap tm_q, const Params p) {
         float m_run = -INFINITY, l_run = 0.f;
         for (int j = 0; alive && j < n_tiles; ++j) {
             const int stage = j & 1;
+            // ---- this thread's 32 keys of tile j: validity bits and (fp8) scales, read
+            // before the scores (the tile's slots and scales are published before its S
+            // is issued, so this wait never delays the one for S)
+            if (!mbar_wait_warp(&meta[stage], (j >> 1) & 1, p.check)) { alive = false; break; }
+            uint32_t valid = 0u;
+            float tsc[kFp8 ? 32 : 1];
+            {
+                const int4* s4 = reinterpret_cast<const int4*>(srow + stage * 64 + 32 * kh);
+#pragma unroll
+                for (int q = 0; q < 8; ++q) {
+                    const int4 v = s4[q];
+                    valid |= (v.x >= 0 ? 1u : 0u) << (4 * q) | (v.y >= 0 ? 2u : 0u) << (4 * q) |
+                             (v.z >= 0 ? 4u : 0u) << (4 * q) | (v.w >= 0 ? 8u : 0u) << (4 * q);
+                }
+                if constexpr (kFp8) {
+                    const float4* c4 = reinterpret_cast<const float4*>(kscale + stage * 64 + 32 * kh);
+#pragma unroll
+                    for (int q = 0; q < 8; ++q) {
+                        const float4 f = c4[q];
+                        tsc[4 * q] = f.x;
+                        tsc[4 * q + 1] = f.y;
+                        tsc[4 * q + 2] = f.z;
+                        tsc[4 * q + 3] = f.w;
+                    }
+                }
+            }
             float x[32];
             {   // ---- scores of tile j: keys 32*kh .. 32*kh+31 of head hl
                 if (!mbar_wait_warp(&sfull[j & 1], (j >> 1) & 1, p.check)) { alive = false; break; }
@@ -660,20 +686,11 @@ mla_pair_kernel(const __grid_constant__ CUtensorMap tm_q, const Params p) {
 #pragma unroll
                 for (int i = 0; i < 32; ++i) x[i] = __uint_as_float(a[i]);
             }
-            if (!mbar_wait_warp(&meta[stage], (j >> 1) & 1, p.check)) { alive = false; break; }
-            const int* ts = srow + stage * 64 + 32 * kh;
-            const float* tsc = kscale + stage * 64 + 32 * kh;
             float sc = p.sc_log2;
             {   // invalid entries (skipped or bad indices) score -inf; fp8 rows x scale
-                const int4* s4 = reinterpret_cast<const int4*>(ts);
 #pragma unroll
-                for (int q = 0; q < 8; ++q) {
-                    const int4 v = s4[q];
-                    if (v.x < 0) x[4 * q] = -INFINITY;
-                    if (v.y < 0) x[4 * q + 1] = -INFINITY;
-                    if (v.z < 0) x[4 * q + 2] = -INFINITY;
-                    if (v.w < 0) x[4 * q + 3] = -INFINITY;
-                }
+                for (int i = 0; i < 32; ++i)
+                    if (!((valid >> i) & 1u)) x[i] = -INFINITY;
                 if constexpr (kFp8) {
 #pragma unroll
                     for (int i = 0; i < 32; ++i) x[i] *= p.sc_log2 * tsc[i];
@@ -707,7 +724,8 @@ mla_pair_kernel(const __grid_constant__ CUtensorMap tm_q, const Params p) {
                 const float e0 = fast_exp2(fmaf(x[i], sc, -msub));
                 const float e1 = fast_exp2(fmaf(x[i + 1], sc, -msub));
                 ls[(i >> 1) & 3] += e0 + e1;
-                pk[i / 2] = kFp8 ? pack_f16(e0 * tsc[i], e1 * tsc[i + 1]) : pack_f16(e0, e1);
+                if constexpr (kFp8) pk[i / 2] = pack_f16(e0 * tsc[i], e1 * tsc[i + 1]);
+                else pk[i / 2] = pack_f16(e0, e1);
             }
             l_run = l_run * alpha + ((ls[0] + ls[1]) + (ls[2] + ls[3]));
             // ---- P_j into P buffer j%2 once P_{j-2}.V has read it
