@@ -352,6 +352,43 @@ indexer_fp8_tc_kernel(const __grid_constant__ CUtensorMap tm_k,
                 // the warp's rows kPair at a time: all their 32-head TMEM loads are issued
                 // before one wait (a TMEM load takes a few hundred cycles; issued one after
                 // another they would serialise that latency)
+                // one row at a time (four warpgroups: no registers for two): each half-row's
+                // 32 accumulator columns and its 32 head weights are loaded together, so
+                // the weights' shared-memory latency overlaps the TMEM load
+                if constexpr (kPair == 1) {
+#pragma unroll
+                    for (int u = 0; u < kRows; ++u) {
+                        if (u >= my_rows) break;
+                        const int qi = q_lo + u;
+                        const uint32_t c0 = tbase + qi * kHeads;
+                        const uint32_t w_sa = smem_u32(w_run + qi * kHeads);
+                        float2 acc[4] = {{0.f, 0.f}, {0.f, 0.f}, {0.f, 0.f}, {0.f, 0.f}};
+#pragma unroll
+                        for (int half = 0; half < 2; ++half) {
+                            uint32_t v[32];
+                            float4 wq[8];
+                            tmem_ld32(c0 + 32 * half, v);
+#pragma unroll
+                            for (int q = 0; q < 8; ++q)   // volatile: see below
+                                asm volatile("ld.shared.v4.f32 {%0, %1, %2, %3}, [%4];"
+                                             : "=f"(wq[q].x), "=f"(wq[q].y), "=f"(wq[q].z), "=f"(wq[q].w)
+                                             : "r"(w_sa + 128 * half + 16 * q));
+                            tmem_ld_wait();
+                            if (half == 1 && u + 1 >= my_rows) release();
+#pragma unroll
+                            for (int q = 0; q < 8; ++q) {
+                                const float2 r0 = make_float2(fmaxf(__uint_as_float(v[4 * q + 0]), 0.f),
+                                                              fmaxf(__uint_as_float(v[4 * q + 1]), 0.f));
+                                const float2 r1 = make_float2(fmaxf(__uint_as_float(v[4 * q + 2]), 0.f),
+                                                              fmaxf(__uint_as_float(v[4 * q + 3]), 0.f));
+                                ffma2(acc[(2 * q) & 3], make_float2(wq[q].x, wq[q].y), r0);
+                                ffma2(acc[(2 * q + 1) & 3], make_float2(wq[q].z, wq[q].w), r1);
+                            }
+                        }
+                        res[u] = ((acc[0].x + acc[0].y) + (acc[1].x + acc[1].y)) +
+                                 ((acc[2].x + acc[2].y) + (acc[3].x + acc[3].y));
+                    }
+                } else {
 #pragma unroll
                 for (int u0 = 0; u0 < kRows; u0 += kPair) {
                     const int nr = min(kPair, my_rows - u0);   // rows of this group
@@ -394,6 +431,7 @@ indexer_fp8_tc_kernel(const __grid_constant__ CUtensorMap tm_k,
                         res[u0 + u] = ((acc[0].x + acc[0].y) + (acc[1].x + acc[1].y)) +
                                       ((acc[2].x + acc[2].y) + (acc[3].x + acc[3].y));
                     }
+                }
                 }
 #pragma unroll
                 for (int u = 0; u < kRows; ++u) {
