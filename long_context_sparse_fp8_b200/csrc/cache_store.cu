@@ -20,11 +20,13 @@
 // The FP8 codes are e4m3(x / scale) with the quotient correctly rounded to fp32.  A
 // division per element would make the kernel compute-bound, so each quotient is first
 // taken as x * (1/scale), which lies within 3 fp32 ulps of the correctly rounded
-// quotient; when the e4m3 codes of that product scaled by (1 - 2^-20) and by
-// (1 + 2^-20) agree, every value in between -- the exact quotient among them -- has the
-// same code (rounding is monotone), and otherwise (a product next to an e4m3 rounding
-// boundary, about one element in 10^5) the code is taken from the division itself.
-// Scales below the smallest normal fp32, whose reciprocal may overflow, divide always.
+// quotient.  In the normal e4m3 range (|q| >= 2^-6) the codes change only at the
+// midpoints between neighbouring e4m3 values, fp32 numbers whose low 20 mantissa bits
+// are 0x80000; a product more than 3 ulps from such a midpoint has the code of the
+// exact quotient (rounding is monotone).  An 8-element chunk with any element within 3
+// ulps of a midpoint, or nonzero below 2^-6 (e4m3 subnormals), takes its codes from the
+// divisions instead (out of line: about one chunk in 10^4 on Gaussian rows).  Scales
+// below the smallest normal fp32, whose reciprocal may overflow, divide always.
 #include <atomic>
 
 #include "common.cuh"
@@ -73,19 +75,39 @@ __device__ __forceinline__ uint32_t e4m3x2(float lo, float hi) {
     return r;
 }
 
-// e4m3 codes of a / sc and b / sc, the quotients correctly rounded to fp32 (see the
-// head of the file); rcp = 1/sc correctly rounded.
-__device__ __forceinline__ uint32_t e4m3x2_div(float a, float b, float sc, float rcp,
-                                               bool divide_all) {
-    if (!divide_all) {
-        const float qa = __fmul_rn(a, rcp), qb = __fmul_rn(b, rcp);
-        const uint32_t code = e4m3x2(qa, qb);
-        const float dn = 1.0f - 0x1p-20f, up = 1.0f + 0x1p-20f;
-        const uint32_t lo = e4m3x2(__fmul_rn(qa, dn), __fmul_rn(qb, dn));
-        const uint32_t hi = e4m3x2(__fmul_rn(qa, up), __fmul_rn(qb, up));
-        if (lo == code && hi == code) return code;
+// e4m3 codes of the 8 quotients f[e] / sc, each correctly rounded to fp32 first: the
+// divisions themselves (the rare path; kept out of line).
+__device__ __noinline__ uint2 e4m3x8_divide(float f0, float f1, float f2, float f3, float f4,
+                                            float f5, float f6, float f7, float sc) {
+    return make_uint2(e4m3x2(__fdiv_rn(f0, sc), __fdiv_rn(f1, sc)) |
+                          (e4m3x2(__fdiv_rn(f2, sc), __fdiv_rn(f3, sc)) << 16),
+                      e4m3x2(__fdiv_rn(f4, sc), __fdiv_rn(f5, sc)) |
+                          (e4m3x2(__fdiv_rn(f6, sc), __fdiv_rn(f7, sc)) << 16));
+}
+
+// Whether the product q = x * (1/sc) may round to another e4m3 code than the correctly
+// rounded quotient (see the head of the file).
+__device__ __forceinline__ bool e4m3_risky(float q) {
+    const uint32_t m = __float_as_uint(q) & 0x7FFFFFFFu;
+    return (m != 0u && m < 0x3C800000u) || ((m & 0xFFFFFu) - 0x7FFFDu) <= 6u;
+}
+
+// e4m3 codes of an 8-element chunk divided by sc (rcp = 1/sc correctly rounded).
+template <int XT>
+__device__ __forceinline__ uint2 e4m3x8_quotients(const Chunk<XT>& c, float sc, float rcp,
+                                                  bool divide_all) {
+    float q[8];
+    bool risky = divide_all;
+#pragma unroll
+    for (int e = 0; e < 8; ++e) {
+        q[e] = __fmul_rn(elem<XT>(c, e), rcp);
+        risky |= e4m3_risky(q[e]);
     }
-    return e4m3x2(__fdiv_rn(a, sc), __fdiv_rn(b, sc));
+    if (risky)
+        return e4m3x8_divide(elem<XT>(c, 0), elem<XT>(c, 1), elem<XT>(c, 2), elem<XT>(c, 3),
+                             elem<XT>(c, 4), elem<XT>(c, 5), elem<XT>(c, 6), elem<XT>(c, 7), sc);
+    return make_uint2(e4m3x2(q[0], q[1]) | (e4m3x2(q[2], q[3]) << 16),
+                      e4m3x2(q[4], q[5]) | (e4m3x2(q[6], q[7]) << 16));
 }
 
 __device__ __forceinline__ uint32_t bf16x2(float lo, float hi) {
@@ -151,12 +173,7 @@ __global__ void __launch_bounds__(kThreads) cache_store_kernel(
                 for (int r = 0; r < CPL; ++r) {
                     const int c = gl + LPR * r;
                     if (c >= nch) continue;
-                    uint32_t q[4];
-#pragma unroll
-                    for (int e = 0; e < 4; ++e)
-                        q[e] = e4m3x2_div(elem<XT>(v[u][r], 2 * e), elem<XT>(v[u][r], 2 * e + 1), sc,
-                                          rcp, divide_all);
-                    *reinterpret_cast<uint2*>(dst + 8 * c) = make_uint2(q[0] | (q[1] << 16), q[2] | (q[3] << 16));
+                    *reinterpret_cast<uint2*>(dst + 8 * c) = e4m3x8_quotients<XT>(v[u][r], sc, rcp, divide_all);
                 }
                 if (gl == 0) scale[slot[u]] = sc;
             } else if constexpr (CT == kBF16) {
