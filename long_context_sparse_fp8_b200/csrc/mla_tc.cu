@@ -687,10 +687,14 @@ mla_pair_kernel(const __grid_constant__ CUtensorMap tm_q, const Params p) {
                 for (int i = 0; i < 32; ++i) x[i] = __uint_as_float(a[i]);
             }
             float sc = p.sc_log2;
-            {   // invalid entries (skipped or bad indices) score -inf; fp8 rows x scale
+            {   // invalid entries (skipped or bad indices) score -inf; fp8 rows x scale.
+                // A warp's lanes share the tile's 32 keys (only the head differs), so
+                // `valid` is warp-uniform and full tiles skip the masking
+                if (valid != 0xFFFFFFFFu) {
 #pragma unroll
-                for (int i = 0; i < 32; ++i)
-                    if (!((valid >> i) & 1u)) x[i] = -INFINITY;
+                    for (int i = 0; i < 32; ++i)
+                        if (!((valid >> i) & 1u)) x[i] = -INFINITY;
+                }
                 if constexpr (kFp8) {
 #pragma unroll
                     for (int i = 0; i < 32; ++i) x[i] *= p.sc_log2 * tsc[i];
