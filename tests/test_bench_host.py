@@ -46,3 +46,24 @@ def test_sparse_attention_ratio_and_store_bytes():
     assert bench.sparse_ratio(spec) == 1.0            # dense fallback: every key attended
     x = types.SimpleNamespace(shape=(131072, 576), element_size=lambda: 2)
     assert bench._store_bytes(x, 1) == 131072 * (1152 + 576 + 4 + 8) == 228_065_280
+
+
+def test_chunked_select_blocks_follow_the_workspace():
+    """The chunked prefill's launch count restates the library's row-block rule: the
+    minimum (L2-sized) workspace gives 148 x 2^m rows per block, a workspace for a whole
+    chunk's logits gives one block per chunk (two stores, one indexer, one top-k and one
+    attention launch per chunk)."""
+    from long_context_sparse_fp8_b200 import chunked as CH
+    Q, L = 8192, 131072
+    assert CH._block_rows(Q, L) == 148                       # 80 MB / (131072 x 4 B) = 160
+    assert CH._block_rows(Q, 8192) == 148 * 16                # 2560 rows fit: 2368
+    assert CH._block_rows(Q, 32768) == 592
+    assert CH._block_rows(Q, L, Q * L * 4) == Q               # the whole chunk
+    assert CH._block_rows(Q, L, 2 * 148 * L * 4 + 100) == 296
+    assert CH._block_rows(100, L, 1) == 100                   # fewer rows than a block
+    cp = types.SimpleNamespace(batches=[types.SimpleNamespace(total_q=Q, max_seq_len=Q * (c + 1))
+                                        for c in range(16)],
+                               ws=types.SimpleNamespace(numel=lambda: Q * L * 4))
+    assert CH.ChunkedPrefill.launches_per_step(cp) == 16 * 5
+    cp.ws = types.SimpleNamespace(numel=lambda: 16)
+    assert CH.ChunkedPrefill.launches_per_step(cp) == 1246
